@@ -78,7 +78,7 @@ def _declare(L):
     L.oracle_e4m3_encode_satfinite.restype = ctypes.c_uint8
     L.oracle_mask_padding.argtypes = [P, I32, I32, I32, I32]
     L.oracle_mask_padding.restype = None
-    L.oracle_create_indices.argtypes = [P, I64, I32, P, P, P, P, P]
+    L.oracle_create_indices.argtypes = [P, I64, I32, P, P, P, P, P, P]
     L.oracle_create_indices.restype = None
     L.oracle_mxfp4_row_stride.argtypes = [I32]
     L.oracle_mxfp4_row_stride.restype = I32
@@ -148,10 +148,12 @@ def create_indices(topk_ids: np.ndarray, E: int) -> dict:
     restore = np.empty(S, np.uint32)
     eids = np.empty(E, np.int32)
     stats = np.empty(2, np.uint32)
+    soff = np.empty(E + 1, np.uint32)
     _load().oracle_create_indices(pid, S, E, _ptr(order), _ptr(start), _ptr(restore),
-                                  _ptr(eids), _ptr(stats))
+                                  _ptr(eids), _ptr(stats), _ptr(soff))
     return dict(token_expert_order=order, expert_start_indices=start,
-                restore_token_order=restore, expert_ids=eids, expert_usage_stats=stats)
+                restore_token_order=restore, expert_ids=eids, expert_usage_stats=stats,
+                scales_offset=soff)
 
 
 # ---------------------------------------------------------------- step 3

@@ -125,12 +125,16 @@ EXPORT void oracle_mask_padding(int64_t *routing_map, int32_t N, int32_t top_k,
 /*                       unrouted pairs = 0xFFFFFFFF                   */
 /*   expert_ids          active experts in ascending id; tail = -1     */
 /*   expert_usage_stats  {max pairs on one expert, active experts}     */
+/*   scales_offset       (optional) offset of each active expert when  */
+/*                       every expert's rows are padded to a multiple  */
+/*                       of 128 ("aligned scale offsets for block-     */
+/*                       scaled grouped matmul"); tail = padded total  */
 /* Ids outside [0, E) (the -1 padding sentinel included) route nowhere.*/
 /* ------------------------------------------------------------------ */
 EXPORT void oracle_create_indices(const int64_t *topk_ids, int64_t S, int32_t E,
                                   uint32_t *token_expert_order, uint32_t *expert_start_indices,
                                   uint32_t *restore_token_order, int32_t *expert_ids,
-                                  uint32_t *expert_usage_stats) {
+                                  uint32_t *expert_usage_stats, uint32_t *scales_offset) {
   uint32_t *cnt = (uint32_t *)calloc((size_t)E, sizeof(uint32_t));
   int32_t A = 0;
   uint32_t maxc = 0, pos = 0;
@@ -164,6 +168,12 @@ EXPORT void oracle_create_indices(const int64_t *topk_ids, int64_t S, int32_t E,
   }
   expert_usage_stats[0] = maxc;
   expert_usage_stats[1] = (uint32_t)A;
+  if (scales_offset) {
+    scales_offset[0] = 0;
+    for (int32_t i = 0; i < A; ++i)
+      scales_offset[i + 1] = scales_offset[i] + (cnt[expert_ids[i]] + 127u) / 128u * 128u;
+    for (int32_t i = A + 1; i <= E; ++i) scales_offset[i] = scales_offset[A];
+  }
   free(cnt);
 }
 

@@ -58,6 +58,11 @@ def check_grouping(ids, E, out):
     # contiguous, ascending-id groups
     grp = ids[out["token_expert_order"][:R].astype(np.int64)]
     assert np.all(np.diff(grp) >= 0)
+    # scales_offset: 128-aligned, each active expert gets its count rounded up
+    so = out["scales_offset"].astype(np.int64)
+    assert np.all(so % 128 == 0) and so[0] == 0
+    np.testing.assert_array_equal(np.diff(so[:A + 1]), -(-cnt[active] // 128) * 128)
+    assert np.all(so[:A + 1] >= start) and np.all(so[A + 1:] == so[A])
 
 
 @pytest.mark.parametrize("S,E,lo", [(0, 4, 0), (1, 1, 0), (32, 8, -1), (257, 5, -2),
