@@ -1,0 +1,351 @@
+// moe_route.cu -- C ABI of the MoE token-routing library (see
+// include/moe_route.h for the contract of every entry point).
+//
+// Host side of each call: validate arguments, check the device is sm_100,
+// choose the kernel variant and launch configuration, enqueue on the
+// caller's stream.  No allocation, no synchronisation (except in
+// moe_get_device_error).
+#include <cstdio>
+#include <cstdlib>
+#include <mutex>
+
+#include "combine.cuh"
+#include "common.cuh"
+#include "create_indices.cuh"
+#include "dispatch_mxfp4.cuh"
+#include "gemv_nvfp4.cuh"
+#include "mask.cuh"
+#include "quant_nvfp4.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  int checked = 0;
+  int supported = 0;
+  int sms = 0;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Current device must be sm_100 (B200 class).  The forced-architecture
+// override exists for host-side tests of the rejection path.
+moe_status_t check_device(int *sms = nullptr) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_dev_mu);
+  DeviceInfo &d = g_dev[dev];
+  if (!d.checked) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return MOE_ERR_CUDA;
+    }
+    const char *force = std::getenv("MOE_FORCE_ARCH");
+    if (force && *force) {
+      major = std::atoi(force) / 10;
+      minor = std::atoi(force) % 10;
+    }
+    d.supported = (major == 10 && minor == 0);
+    d.sms = sms;
+    d.checked = 1;
+  }
+  if (!d.supported) return MOE_ERR_UNSUPPORTED_ARCH;
+  if (sms) *sms = d.sms;
+  return MOE_OK;
+}
+
+moe_status_t launch_status() {
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+template <typename Kernel>
+moe_status_t set_smem(Kernel k, size_t bytes) {
+  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
+int64_t tiles_for(int64_t S) { return (S + moe::idx::kTileSlots - 1) / moe::idx::kTileSlots; }
+
+}  // namespace
+
+extern "C" {
+
+int32_t moe_version(void) { return 100; }
+
+const char *moe_status_string(moe_status_t st) {
+  switch (st) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED_ARCH: return "unsupported architecture (sm_100 required)";
+    case MOE_ERR_WORKSPACE: return "workspace missing or too small";
+    case MOE_ERR_CUDA: return "CUDA error";
+  }
+  return "unknown status";
+}
+
+moe_status_t moe_get_device_error(uint32_t *host_flags, int32_t clear) {
+  if (!host_flags) return MOE_ERR_INVALID_ARG;
+  moe_status_t st = check_device();
+  if (st != MOE_OK) return st;
+  if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaMemcpyFromSymbol(host_flags, moe::g_device_error, sizeof(uint32_t)) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (clear) {
+    const uint32_t zero = 0;
+    if (cudaMemcpyToSymbol(moe::g_device_error, &zero, sizeof(uint32_t)) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
+// ------------------------------------------------------------------ step 1
+moe_status_t moe_mask_padding(int64_t *routing_map, int32_t N, int32_t top_k,
+                              const int32_t *real_token_count, int32_t tp_rank, cudaStream_t s) {
+  if (N < 0 || top_k < 1 || tp_rank < 0 || !real_token_count) return MOE_ERR_INVALID_ARG;
+  if (N > 0 && !routing_map) return MOE_ERR_INVALID_ARG;
+  if (!aligned(routing_map, 8) || !aligned(real_token_count, 4)) return MOE_ERR_INVALID_ARG;
+  int sms = 0;
+  moe_status_t st = check_device(&sms);
+  if (st != MOE_OK) return st;
+  if (N == 0) return MOE_OK;
+  const int64_t slots = (int64_t)N * top_k;
+  int64_t blocks = (slots + 255) / 256;
+  if (blocks > (int64_t)sms * 8) blocks = (int64_t)sms * 8;
+  moe::mask_padding_kernel<<<(unsigned)blocks, 256, 0, s>>>(routing_map, N, top_k,
+                                                             real_token_count, tp_rank);
+  return launch_status();
+}
+
+// ------------------------------------------------------------------ step 2
+size_t moe_create_indices_workspace_bytes(int64_t num_slots, int32_t E) {
+  if (num_slots <= moe::idx::kSmallSlots || E < 1) return moe::idx::kWsHeader;
+  return moe::idx::kWsHeader + (size_t)tiles_for(num_slots) * (size_t)E * sizeof(uint32_t);
+}
+
+moe_status_t moe_create_indices(const int64_t *topk_ids, int64_t num_slots, int32_t E,
+                                uint32_t *token_expert_order, uint32_t *expert_start_indices,
+                                uint32_t *restore_token_order, int32_t *expert_ids,
+                                uint32_t *expert_usage_stats, uint32_t *scales_offset,
+                                void *workspace, size_t ws_bytes, cudaStream_t s) {
+  using namespace moe::idx;
+  if (E < 1 || E > 1024 || num_slots < 0 || num_slots >= (int64_t(1) << 31))
+    return MOE_ERR_INVALID_ARG;
+  if (!expert_start_indices || !expert_ids || !expert_usage_stats) return MOE_ERR_INVALID_ARG;
+  if (num_slots > 0 && (!topk_ids || !token_expert_order || !restore_token_order))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned(topk_ids, 8) || !aligned(token_expert_order, 4) ||
+      !aligned(restore_token_order, 4) || !aligned(expert_start_indices, 4) ||
+      !aligned(expert_ids, 4) || !aligned(expert_usage_stats, 4) || !aligned(scales_offset, 4))
+    return MOE_ERR_INVALID_ARG;
+  const size_t need = moe_create_indices_workspace_bytes(num_slots, E);
+  if (!workspace || ws_bytes < need || !aligned(workspace, 256)) return MOE_ERR_WORKSPACE;
+  moe_status_t st = check_device();
+  if (st != MOE_OK) return st;
+  const size_t smem = smem_bytes(E);
+  if (num_slots <= kSmallSlots) {
+    if ((st = set_smem(create_indices_small_kernel, smem)) != MOE_OK) return st;
+    create_indices_small_kernel<<<1, kThreads, smem, s>>>(
+        topk_ids, num_slots, E, token_expert_order, expert_start_indices, restore_token_order,
+        expert_ids, expert_usage_stats, scales_offset);
+    return launch_status();
+  }
+  const int64_t T = tiles_for(num_slots);
+  uint32_t *ticket = static_cast<uint32_t *>(workspace);
+  uint32_t *tiles = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(workspace) + kWsHeader);
+  if (cudaMemsetAsync(ticket, 0, sizeof(uint32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
+  if ((st = set_smem(create_indices_hist_kernel, smem)) != MOE_OK) return st;
+  if ((st = set_smem(create_indices_scatter_kernel, smem)) != MOE_OK) return st;
+  create_indices_hist_kernel<<<(unsigned)T, kThreads, smem, s>>>(
+      topk_ids, num_slots, E, token_expert_order, expert_start_indices, expert_ids,
+      expert_usage_stats, scales_offset, ticket, tiles);
+  if ((st = launch_status()) != MOE_OK) return st;
+  create_indices_scatter_kernel<<<(unsigned)T, kThreads, smem, s>>>(
+      topk_ids, num_slots, E, token_expert_order, restore_token_order, tiles);
+  return launch_status();
+}
+
+// ------------------------------------------------------------------ step 3
+size_t moe_mxfp4_row_stride(int32_t K) {
+  if (K <= 0) return 0;
+  const size_t raw = (size_t)K / 2 + (size_t)K / 32;
+  return (raw + 15) / 16 * 16;
+}
+
+moe_status_t moe_dispatch_mxfp4(const void *input_tokens, int32_t N, int32_t K, int32_t top_k,
+                                int32_t E, const uint32_t *restore_token_order,
+                                const uint32_t *expert_start_indices, const int32_t *expert_ids,
+                                const uint32_t *expert_usage_stats, uint8_t *recv_buf,
+                                int64_t recv_capacity, uint32_t *recv_counts, cudaStream_t s) {
+  if (N < 0 || K <= 0 || K % 32 != 0 || top_k < 1 || E < 1 || E > 1024 || top_k > E ||
+      recv_capacity < 0)
+    return MOE_ERR_INVALID_ARG;
+  if (!expert_start_indices || !expert_ids || !expert_usage_stats || !recv_counts)
+    return MOE_ERR_INVALID_ARG;
+  if (N > 0 && (!input_tokens || !restore_token_order)) return MOE_ERR_INVALID_ARG;
+  if (recv_capacity > 0 && !recv_buf) return MOE_ERR_INVALID_ARG;
+  if (!aligned(input_tokens, 16) || !aligned(recv_buf, 16) || !aligned(recv_counts, 4))
+    return MOE_ERR_INVALID_ARG;
+  int sms = 0;
+  moe_status_t st = check_device(&sms);
+  if (st != MOE_OK) return st;
+  const int wpb = moe::disp::kWarpsPerBlock;
+  int64_t blocks = ((int64_t)N + wpb - 1) / wpb;
+  if (blocks < 1) blocks = 1;
+  if (blocks > (int64_t)sms * 16) blocks = (int64_t)sms * 16;
+  moe::disp::dispatch_mxfp4_kernel<<<(unsigned)blocks, wpb * 32, 0, s>>>(
+      static_cast<const uint16_t *>(input_tokens), N, K, top_k, E, restore_token_order,
+      expert_start_indices, expert_ids, expert_usage_stats, recv_buf, recv_capacity,
+      (int32_t)moe_mxfp4_row_stride(K), recv_counts);
+  return launch_status();
+}
+
+// ------------------------------------------------------------------ step 4a
+moe_status_t moe_quantize_activations_nvfp4(const void *x, int32_t M, int32_t K,
+                                            float act_global, uint8_t *xq, uint8_t *sfa,
+                                            cudaStream_t s) {
+  if (M < 0 || K <= 0 || K % 16 != 0 || !(act_global > 0.0f)) return MOE_ERR_INVALID_ARG;
+  if (M > 0 && (!x || !xq || !sfa)) return MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(xq, 4)) return MOE_ERR_INVALID_ARG;
+  int sms = 0;
+  moe_status_t st = check_device(&sms);
+  if (st != MOE_OK) return st;
+  if (M == 0) return MOE_OK;
+  const int wpb = moe::nvq::kWarpsPerBlock;
+  const int64_t work = (int64_t)M * ((K + 255) / 256);
+  int64_t blocks = (work + wpb - 1) / wpb;
+  if (blocks > (int64_t)sms * 16) blocks = (int64_t)sms * 16;
+  moe::nvq::quant_act_nvfp4_kernel<<<(unsigned)blocks, wpb * 32, 0, s>>>(
+      static_cast<const uint16_t *>(x), M, K, act_global, xq, sfa);
+  return launch_status();
+}
+
+moe_status_t moe_quantize_weights_nvfp4(const float *w, int32_t E, int32_t N, int32_t K,
+                                        uint8_t *wq, uint8_t *sfw, float *w_global,
+                                        cudaStream_t s) {
+  if (E < 1 || N < 1 || K <= 0 || K % 16 != 0) return MOE_ERR_INVALID_ARG;
+  if (!w || !wq || !sfw || !w_global) return MOE_ERR_INVALID_ARG;
+  if (!aligned(w, 16) || !aligned(wq, 4) || !aligned(w_global, 4)) return MOE_ERR_INVALID_ARG;
+  int sms = 0;
+  moe_status_t st = check_device(&sms);
+  if (st != MOE_OK) return st;
+  if (cudaMemsetAsync(w_global, 0, sizeof(float) * (size_t)E, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  const int64_t per_expert = (int64_t)N * K;
+  int64_t cx = (per_expert + 256 * 64 - 1) / (256 * 64);
+  if (cx > 1024) cx = 1024;
+  moe::nvq::weight_amax_kernel<<<dim3((unsigned)cx, (unsigned)E), 256, 0, s>>>(
+      w, per_expert, reinterpret_cast<unsigned int *>(w_global));
+  if ((st = launch_status()) != MOE_OK) return st;
+  const int wpb = moe::nvq::kWarpsPerBlock;
+  const int64_t work = (int64_t)E * N * ((K + 255) / 256);
+  int64_t blocks = (work + wpb - 1) / wpb;
+  if (blocks > (int64_t)sms * 32) blocks = (int64_t)sms * 32;
+  moe::nvq::quant_weight_nvfp4_kernel<<<(unsigned)blocks, wpb * 32, 0, s>>>(
+      w, E, N, K, reinterpret_cast<const unsigned int *>(w_global), wq, sfw);
+  if ((st = launch_status()) != MOE_OK) return st;
+  moe::nvq::weight_global_kernel<<<(E + 255) / 256, 256, 0, s>>>(w_global, E);
+  return launch_status();
+}
+
+// ------------------------------------------------------------------ step 4b
+moe_status_t moe_grouped_gemv_nvfp4(moe_gemv_mode_t mode, const void *act, const uint8_t *sfa,
+                                    float act_global, int32_t M, int32_t top_k,
+                                    const uint8_t *w, const uint8_t *sfw, const float *w_global,
+                                    int32_t E, int32_t N, int32_t K,
+                                    const uint32_t *token_expert_order,
+                                    const uint32_t *expert_start_indices,
+                                    const int32_t *expert_ids,
+                                    const uint32_t *expert_usage_stats, void *out,
+                                    cudaStream_t s) {
+  using namespace moe::gemv;
+  if (mode != MOE_W4A16 && mode != MOE_W4A4) return MOE_ERR_INVALID_ARG;
+  if (M < 0 || top_k < 1 || E < 1 || E > kMaxExperts || top_k > E || N < 8 || N % 8 != 0 ||
+      K < 64 || K % 64 != 0 || !(act_global > 0.0f))
+    return MOE_ERR_INVALID_ARG;
+  if (!w || !sfw || !expert_start_indices || !expert_ids || !expert_usage_stats)
+    return MOE_ERR_INVALID_ARG;
+  if (M > 0 && (!act || !out || !token_expert_order)) return MOE_ERR_INVALID_ARG;
+  if (mode == MOE_W4A4 && M > 0 && !sfa) return MOE_ERR_INVALID_ARG;
+  if (!aligned(act, 16) || !aligned(w, 16) || !aligned(sfw, 16) || !aligned(out, 16) ||
+      !aligned(w_global, 4))
+    return MOE_ERR_INVALID_ARG;
+  // the flat unit count must fit 32 bits: (S / 32 + E) * ceil(N / 16)
+  const int64_t S = (int64_t)M * top_k;
+  if ((S / kTS + E + 1) * ((N + 15) / 16) >= (int64_t(1) << 32)) return MOE_ERR_INVALID_ARG;
+  int sms = 0;
+  moe_status_t st = check_device(&sms);
+  if (st != MOE_OK) return st;
+  if (M == 0) return MOE_OK;
+  Params p;
+  p.act = act;
+  p.sfa = sfa;
+  p.g_a = act_global;
+  p.top_k = top_k;
+  p.w = w;
+  p.sfw = sfw;
+  p.w_global = w_global;
+  p.N = N;
+  p.K = K;
+  p.order = token_expert_order;
+  p.start = expert_start_indices;
+  p.eids = expert_ids;
+  p.stats = expert_usage_stats;
+  p.out = static_cast<uint16_t *>(out);
+  const bool sf_bulk = (K % 256) == 0;
+  void (*kern)(const Params);
+  if (mode == MOE_W4A16)
+    kern = sf_bulk ? grouped_gemv_kernel<MOE_W4A16, true> : grouped_gemv_kernel<MOE_W4A16, false>;
+  else
+    kern = sf_bulk ? grouped_gemv_kernel<MOE_W4A4, true> : grouped_gemv_kernel<MOE_W4A4, false>;
+  if ((st = set_smem(kern, kSmemBytes)) != MOE_OK) return st;
+  kern<<<(unsigned)sms, kThreads, kSmemBytes, s>>>(p);
+  return launch_status();
+}
+
+// ------------------------------------------------------------------ step 5
+moe_status_t moe_combine(const void *expert_out, const float *router_weights,
+                         const int64_t *topk_ids, int32_t M, int32_t top_k, int32_t H, int32_t E,
+                         moe_epilogue_t epi, float alpha, void *output_tokens, cudaStream_t s) {
+  if (M < 0 || top_k < 1 || H < 8 || H % 8 != 0 || E < 1) return MOE_ERR_INVALID_ARG;
+  if (epi != MOE_EPI_NONE && epi != MOE_EPI_IDENTITY && epi != MOE_EPI_SCALE)
+    return MOE_ERR_INVALID_ARG;
+  if (M > 0 && (!expert_out || !router_weights || !topk_ids || !output_tokens))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned(expert_out, 16) || !aligned(output_tokens, 16) || !aligned(router_weights, 4) ||
+      !aligned(topk_ids, 8))
+    return MOE_ERR_INVALID_ARG;
+  int sms = 0;
+  moe_status_t st = check_device(&sms);
+  if (st != MOE_OK) return st;
+  if (M == 0) return MOE_OK;
+  const int wpb = moe::comb::kWarpsPerBlock;
+  const int64_t work = (int64_t)M * ((H + 255) / 256);
+  int64_t blocks = (work + wpb - 1) / wpb;
+  if (blocks > (int64_t)sms * 16) blocks = (int64_t)sms * 16;
+  const uint16_t *y = static_cast<const uint16_t *>(expert_out);
+  uint16_t *o = static_cast<uint16_t *>(output_tokens);
+  if (epi == MOE_EPI_SCALE)
+    moe::comb::combine_kernel<MOE_EPI_SCALE><<<(unsigned)blocks, wpb * 32, 0, s>>>(
+        y, router_weights, topk_ids, M, top_k, H, E, alpha, o);
+  else
+    moe::comb::combine_kernel<MOE_EPI_IDENTITY><<<(unsigned)blocks, wpb * 32, 0, s>>>(
+        y, router_weights, topk_ids, M, top_k, H, E, alpha, o);
+  return launch_status();
+}
+
+}  // extern "C"

@@ -1,0 +1,137 @@
+"""Buffer owner for one single-GPU routing step: torch allocates device memory,
+the library's kernels do all the work.
+
+    pipe = RoutingPipeline(N=128, K=2048, E=128, top_k=8, N_out=768, mode="w4a16")
+    pipe.quantize_weights(w_f32_expert_slices)      # offline, once
+    pipe.x.copy_(...); pipe.routing_map.copy_(...); pipe.router_weights.copy_(...)
+    pipe.real_token_count.fill_(real)
+    pipe.run()                                      # mask -> indices -> dispatch -> GEMV -> combine
+    pipe.output                                     # bf16 [N, N_out]
+
+Every buffer is allocated once at construction, so ``run`` allocates
+nothing and can be captured in a CUDA graph.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import (MOE_EPI_IDENTITY, MOE_EPI_NONE, MOE_EPI_SCALE, MOE_W4A4, MOE_W4A16,
+               moe_combine, moe_create_indices, moe_create_indices_workspace_bytes,
+               moe_dispatch_mxfp4, moe_grouped_gemv_nvfp4, moe_mask_padding,
+               moe_mxfp4_row_stride, moe_quantize_activations_nvfp4, moe_quantize_weights_nvfp4)
+
+EPILOGUES = {"none": MOE_EPI_NONE, "identity": MOE_EPI_IDENTITY, "scale": MOE_EPI_SCALE}
+
+
+class RoutingPipeline:
+    def __init__(self, N: int, K: int, E: int, top_k: int, N_out: int, mode: str = "w4a16",
+                 epilogue: str = "none", alpha: float = 1.0, tp_rank: int = 0,
+                 act_global: float = 1.0, device: str | torch.device = "cuda",
+                 recv_capacity: int | None = None, dispatch: bool = True):
+        self.N, self.K, self.E, self.top_k, self.N_out = N, K, E, top_k, N_out
+        self.mode = mode
+        self.gemv_mode = MOE_W4A16 if mode == "w4a16" else MOE_W4A4
+        self.epi = EPILOGUES[epilogue]
+        self.alpha = float(alpha)
+        self.tp_rank = tp_rank
+        self.act_global = float(act_global)
+        self.dispatch = dispatch
+        dev = torch.device(device)
+        self.device = dev
+        S = N * top_k
+        self.S = S
+        u8, i32, i64 = torch.uint8, torch.int32, torch.int64
+        # inputs
+        self.x = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
+        self.routing_map = torch.empty((N, top_k), dtype=i64, device=dev)
+        self.router_weights = torch.empty((N, top_k), dtype=torch.float32, device=dev)
+        self.real_token_count = torch.zeros(1, dtype=i32, device=dev)
+        # expert library
+        self.wq = torch.empty((E, N_out, K // 2), dtype=u8, device=dev)
+        self.sfw = torch.empty((E, N_out, K // 16), dtype=u8, device=dev)
+        self.w_global = torch.ones(E, dtype=torch.float32, device=dev)
+        # step 2
+        self.token_expert_order = torch.empty(S, dtype=i32, device=dev)
+        self.expert_start_indices = torch.empty(E + 1, dtype=i32, device=dev)
+        self.restore_token_order = torch.empty(S, dtype=i32, device=dev)
+        self.expert_ids = torch.empty(E, dtype=i32, device=dev)
+        self.expert_usage_stats = torch.empty(2, dtype=i32, device=dev)
+        self.scales_offset = torch.empty(E + 1, dtype=i32, device=dev)
+        self.ws_bytes = moe_create_indices_workspace_bytes(S, E)
+        self.workspace = torch.empty(max(self.ws_bytes, 256), dtype=u8, device=dev)
+        # step 3
+        self.stride = moe_mxfp4_row_stride(K)
+        self.recv_capacity = S if recv_capacity is None else recv_capacity
+        self.recv_buf = torch.empty((self.recv_capacity, self.stride), dtype=u8, device=dev)
+        self.recv_counts = torch.empty(E, dtype=i32, device=dev)
+        # step 4
+        if self.gemv_mode == MOE_W4A4:
+            self.xq = torch.empty((N, K // 2), dtype=u8, device=dev)
+            self.sfa = torch.empty((N, K // 16), dtype=u8, device=dev)
+        else:
+            self.xq = self.sfa = None
+        self.expert_out = torch.zeros((N, top_k, N_out), dtype=torch.bfloat16, device=dev)
+        # step 5
+        self.output = torch.empty((N, N_out), dtype=torch.bfloat16, device=dev)
+
+    # ------------------------------------------------------------ weights
+    def quantize_weights(self, w_f32: torch.Tensor, expert_base: int = 0, stream=None):
+        """Quantise fp32 weights [e, N_out, K] (device) into experts [base, base + e)."""
+        e = w_f32.shape[0]
+        assert w_f32.shape[1:] == (self.N_out, self.K) and w_f32.is_cuda
+        w = w_f32.contiguous()
+        moe_quantize_weights_nvfp4(w, e, self.N_out, self.K, self.wq[expert_base:expert_base + e],
+                                   self.sfw[expert_base:expert_base + e],
+                                   self.w_global[expert_base:expert_base + e], stream)
+
+    # ------------------------------------------------------------ steps
+    def mask(self, stream=None):
+        moe_mask_padding(self.routing_map, self.N, self.top_k, self.real_token_count,
+                         self.tp_rank, stream)
+
+    def create_indices(self, stream=None):
+        moe_create_indices(self.routing_map, self.S, self.E, self.token_expert_order,
+                           self.expert_start_indices, self.restore_token_order, self.expert_ids,
+                           self.expert_usage_stats, self.scales_offset, self.workspace,
+                           self.ws_bytes, stream)
+
+    def dispatch_mxfp4(self, stream=None):
+        moe_dispatch_mxfp4(self.x, self.N, self.K, self.top_k, self.E, self.restore_token_order,
+                           self.expert_start_indices, self.expert_ids, self.expert_usage_stats,
+                           self.recv_buf, self.recv_capacity, self.recv_counts, stream)
+
+    def quantize_activations(self, stream=None):
+        moe_quantize_activations_nvfp4(self.x, self.N, self.K, self.act_global, self.xq,
+                                       self.sfa, stream)
+
+    def gemv(self, stream=None):
+        act = self.x if self.gemv_mode == MOE_W4A16 else self.xq
+        moe_grouped_gemv_nvfp4(self.gemv_mode, act, self.sfa, self.act_global, self.N,
+                               self.top_k, self.wq, self.sfw, self.w_global, self.E, self.N_out,
+                               self.K, self.token_expert_order, self.expert_start_indices,
+                               self.expert_ids, self.expert_usage_stats, self.expert_out, stream)
+
+    def combine(self, stream=None):
+        moe_combine(self.expert_out, self.router_weights, self.routing_map, self.N, self.top_k,
+                    self.N_out, self.E, self.epi, self.alpha, self.output, stream)
+
+    def run(self, stream=None, gemv_events=None):
+        """All steps in order on one stream.  ``gemv_events`` = (start, end) CUDA
+        events recorded around the GEMV launch, for per-kernel timing."""
+        self.mask(stream)
+        self.create_indices(stream)
+        if self.dispatch:
+            self.dispatch_mxfp4(stream)
+        if self.gemv_mode == MOE_W4A4:
+            self.quantize_activations(stream)
+        if gemv_events is not None:
+            gemv_events[0].record(stream)
+        self.gemv(stream)
+        if gemv_events is not None:
+            gemv_events[1].record(stream)
+        self.combine(stream)
+
+    def launches_per_run(self) -> int:
+        n = 1 + (1 if self.S <= 16384 else 2) + (1 if self.dispatch else 0)
+        n += 1 if self.gemv_mode == MOE_W4A4 else 0
+        return n + 2

@@ -1,0 +1,84 @@
+"""Shared helpers for the GPU parity tests (torch <-> numpy marshalling, tolerances)."""
+import numpy as np
+import torch
+
+import oracle
+import workloads as wl
+
+
+def dev(a: np.ndarray) -> torch.Tensor:
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.uint32:
+        a = a.view(np.int32)
+    if a.dtype == np.uint16:
+        return torch.from_numpy(a.view(np.int16)).cuda().view(torch.bfloat16)
+    return torch.from_numpy(a).cuda()
+
+
+def host_u32(t: torch.Tensor) -> np.ndarray:
+    return t.cpu().numpy().view(np.uint32)
+
+
+def host_bf16_bits(t: torch.Tensor) -> np.ndarray:
+    return t.view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def host_bf16_f64(t: torch.Tensor) -> np.ndarray:
+    return wl.bf16_bits_to_f32(host_bf16_bits(t)).astype(np.float64)
+
+
+def float_tol(ref: np.ndarray) -> np.ndarray:
+    """Per-element bound for fp outputs: 5e-3 relative above a 1e-3 floor."""
+    return np.maximum(1e-3, 5e-3 * np.abs(ref))
+
+
+def assert_float_parity(gpu: np.ndarray, ref: np.ndarray, extra: np.ndarray | float = 0.0,
+                        what: str = ""):
+    gpu = np.asarray(gpu, np.float64)
+    ref = np.asarray(ref, np.float64)
+    err = np.abs(gpu - ref)
+    bound = float_tol(ref) + extra
+    bad = ~(err <= bound)
+    if bad.any():
+        i = np.flatnonzero(bad.ravel())[:5]
+        raise AssertionError(
+            f"{what}: {bad.sum()} / {bad.size} elements out of tolerance; first gpu="
+            f"{gpu.ravel()[i]}, ref={ref.ravel()[i]}, bound={np.broadcast_to(bound, ref.shape).ravel()[i]}")
+
+
+def check_indices(gpu: dict, ref: dict, S: int):
+    for k in ("token_expert_order", "restore_token_order", "expert_start_indices",
+              "expert_usage_stats", "scales_offset"):
+        np.testing.assert_array_equal(gpu[k], ref[k], err_msg=k)
+    np.testing.assert_array_equal(gpu["expert_ids"], ref["expert_ids"], err_msg="expert_ids")
+
+
+def pipeline_indices(pipe) -> dict:
+    return dict(
+        token_expert_order=host_u32(pipe.token_expert_order),
+        expert_start_indices=host_u32(pipe.expert_start_indices),
+        restore_token_order=host_u32(pipe.restore_token_order),
+        expert_ids=pipe.expert_ids.cpu().numpy(),
+        expert_usage_stats=host_u32(pipe.expert_usage_stats),
+        scales_offset=host_u32(pipe.scales_offset),
+    )
+
+
+def load_inputs(pipe, cfg, x_bits, ids, rw):
+    pipe.x.copy_(dev(x_bits))
+    pipe.routing_map.copy_(dev(ids))
+    pipe.router_weights.copy_(dev(rw))
+    pipe.real_token_count.fill_(cfg.real)
+
+
+def quantize_all_weights(pipe, cfg, chunk: int = 16):
+    """GPU-quantise the seeded fp32 weights of every expert, a few at a time."""
+    for e0 in range(0, cfg.E, chunk):
+        es = list(range(e0, min(cfg.E, e0 + chunk)))
+        w = torch.from_numpy(wl.expert_weights_f32_many(cfg, es)).cuda()
+        pipe.quantize_weights(w, expert_base=e0)
+        torch.cuda.synchronize()
+
+
+def oracle_weights(cfg, experts):
+    return oracle.quantize_weights_nvfp4(wl.expert_weights_f32_many(cfg, experts))

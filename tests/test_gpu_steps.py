@@ -1,0 +1,337 @@
+"""GPU parity, step by step: every kernel against the CPU oracle on the same
+seeded inputs, through the C ABI (Python binding).  Bit-exact for indices,
+counts, FP4 codes and E8M0 / E4M3 scales; fp outputs within
+max(1e-3, 5e-3 * |ref|) of the oracle's unrounded fp64 value."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import permute_fp4_dispatch_b200 as moe
+import workloads as wl
+from permute_fp4_dispatch_b200.build import build
+from permute_fp4_dispatch_b200.pipeline import RoutingPipeline
+from tests.gpu_helpers import (assert_float_parity, check_indices, dev, host_bf16_bits,
+                               host_bf16_f64, host_u32, load_inputs, oracle_weights,
+                               pipeline_indices, quantize_all_weights)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def cuda_library():
+    build()
+    moe.library()
+    yield
+    assert moe.moe_get_device_error(clear=True) == 0
+
+
+# ------------------------------------------------------------------ step 1
+@pytest.mark.parametrize("N,k,real,tp", [(16, 2, 13, 0), (640, 8, 512, 0), (4096, 4, 3000, 0),
+                                         (16, 2, 0, 0), (16, 2, -3, 0), (16, 2, 99, 0),
+                                         (10, 3, 25, 2), (10, 3, 15, 1), (1, 1, 0, 0)])
+def test_mask_parity(N, k, real, tp):
+    rng = np.random.default_rng(N + real)
+    m = rng.integers(-2, 50, (N, k)).astype(np.int64)
+    t = dev(m)
+    cnt = torch.tensor([real], dtype=torch.int32, device="cuda")
+    moe.moe_mask_padding(t, N, k, cnt, tp)
+    np.testing.assert_array_equal(t.cpu().numpy(), oracle.mask_padding(m, real, tp))
+
+
+# ------------------------------------------------------------------ step 2
+def gpu_create_indices(ids: np.ndarray, E: int) -> dict:
+    S = ids.size
+    order = torch.empty(max(S, 1), dtype=torch.int32, device="cuda")
+    restore = torch.empty(max(S, 1), dtype=torch.int32, device="cuda")
+    start = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    eids = torch.empty(E, dtype=torch.int32, device="cuda")
+    stats = torch.empty(2, dtype=torch.int32, device="cuda")
+    soff = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    ws_bytes = moe.moe_create_indices_workspace_bytes(S, E)
+    ws = torch.full((ws_bytes,), 0x5A, dtype=torch.uint8, device="cuda")
+    t = dev(ids.reshape(-1).astype(np.int64)) if S else torch.empty(1, dtype=torch.int64,
+                                                                     device="cuda")
+    moe.moe_create_indices(t, S, E, order, start, restore, eids, stats, soff, ws, ws_bytes)
+    out = dict(token_expert_order=host_u32(order)[:S], expert_start_indices=host_u32(start),
+               restore_token_order=host_u32(restore)[:S], expert_ids=eids.cpu().numpy(),
+               expert_usage_stats=host_u32(stats), scales_offset=host_u32(soff))
+    return out
+
+
+@pytest.mark.parametrize("S,E,lo", [(0, 4, 0), (1, 1, 0), (32, 8, -1), (1000, 5, -2),
+                                    (1024, 128, 0), (5120, 256, -1), (16384, 128, -1),
+                                    (16385, 64, 0), (40000, 64, -1), (98304, 64, 0),
+                                    (50000, 1024, -3), (200000, 7, -1)])
+def test_create_indices_parity(S, E, lo):
+    rng = np.random.default_rng(S * 7 + E)
+    ids = rng.integers(lo, E + 2, S).astype(np.int64)
+    check_indices(gpu_create_indices(ids, E), oracle.create_indices(ids, E), S)
+
+
+def test_create_indices_deterministic_and_skewed():
+    rng = np.random.default_rng(3)
+    # heavy skew: one expert takes most slots (tiled path)
+    ids = np.where(rng.random(60000) < 0.9, 5, rng.integers(0, 64, 60000)).astype(np.int64)
+    ref = oracle.create_indices(ids, 64)
+    for _ in range(5):
+        check_indices(gpu_create_indices(ids, 64), ref, ids.size)
+
+
+# ------------------------------------------------------------------ codecs (exhaustive)
+def all_finite_bf16(shuffle_seed=None) -> np.ndarray:
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    bits = bits[((bits >> 7) & 0xFF) != 0xFF]          # drop Inf / NaN
+    if shuffle_seed is not None:
+        bits = np.random.default_rng(shuffle_seed).permutation(bits)
+    n = -(-bits.size // 256) * 256
+    out = np.zeros(n, np.uint16)
+    out[: bits.size] = bits
+    return out.reshape(-1, 256)
+
+
+def gpu_mxfp4_rows(x_bits: np.ndarray) -> np.ndarray:
+    N, K = x_bits.shape
+    ids = np.zeros((N, 1), np.int64)                    # every token to expert 0, in order
+    idx = gpu_tensors_indices(ids, 1)
+    stride = moe.moe_mxfp4_row_stride(K)
+    recv = torch.full((N, stride), 0xA5, dtype=torch.uint8, device="cuda")
+    counts = torch.empty(1, dtype=torch.int32, device="cuda")
+    moe.moe_dispatch_mxfp4(dev(x_bits), N, K, 1, 1, idx["restore"], idx["start"], idx["eids"],
+                           idx["stats"], recv, N, counts)
+    return recv.cpu().numpy()
+
+
+def gpu_tensors_indices(ids: np.ndarray, E: int) -> dict:
+    S = ids.size
+    r = dict(order=torch.empty(S, dtype=torch.int32, device="cuda"),
+             restore=torch.empty(S, dtype=torch.int32, device="cuda"),
+             start=torch.empty(E + 1, dtype=torch.int32, device="cuda"),
+             eids=torch.empty(E, dtype=torch.int32, device="cuda"),
+             stats=torch.empty(2, dtype=torch.int32, device="cuda"))
+    ws_bytes = moe.moe_create_indices_workspace_bytes(S, E)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+    moe.moe_create_indices(dev(ids.reshape(-1)), S, E, r["order"], r["start"], r["restore"],
+                           r["eids"], r["stats"], None, ws, ws_bytes)
+    return r
+
+
+@pytest.mark.parametrize("seed", [None, 1, 2])
+def test_mxfp4_exhaustive_bf16(seed):
+    x = all_finite_bf16(seed)
+    np.testing.assert_array_equal(gpu_mxfp4_rows(x), oracle.mxfp4_encode_rows(x))
+
+
+@pytest.mark.parametrize("K", [32, 96, 2048, 7168 + 32])
+def test_mxfp4_rows_random_scales(K):
+    rng = np.random.default_rng(K)
+    x = (rng.standard_normal((37, K)) * np.exp(rng.uniform(-30, 30, (37, 1)))).astype(np.float32)
+    x[0, :64] = 0.0
+    x[1, :32] = -0.0
+    xb = wl.f32_to_bf16_bits(x)
+    np.testing.assert_array_equal(gpu_mxfp4_rows(xb), oracle.mxfp4_encode_rows(xb))
+
+
+def gpu_nvfp4_act(x_bits: np.ndarray, g: float):
+    M, K = x_bits.shape
+    xq = torch.empty((M, K // 2), dtype=torch.uint8, device="cuda")
+    sfa = torch.empty((M, K // 16), dtype=torch.uint8, device="cuda")
+    moe.moe_quantize_activations_nvfp4(dev(x_bits), M, K, g, xq, sfa)
+    return xq.cpu().numpy(), sfa.cpu().numpy()
+
+
+@pytest.mark.parametrize("seed,g", [(None, 1.0), (1, 1.0), (2, 0.37), (None, 3.5e-3)])
+def test_nvfp4_activation_exhaustive_bf16(seed, g):
+    x = all_finite_bf16(seed)
+    g = float(np.float32(g))
+    q, s = gpu_nvfp4_act(x, g)
+    rq, rs = oracle.nvfp4_quantize_bf16(x, g)
+    np.testing.assert_array_equal(s, rs)
+    np.testing.assert_array_equal(q, rq)
+
+
+@pytest.mark.parametrize("M,K", [(5, 16), (33, 2880), (3, 4096 + 16)])
+def test_nvfp4_activation_shapes(M, K):
+    rng = np.random.default_rng(M * K)
+    xb = wl.f32_to_bf16_bits((rng.standard_normal((M, K)) * 3).astype(np.float32))
+    q, s = gpu_nvfp4_act(xb, 1.0)
+    rq, rs = oracle.nvfp4_quantize_bf16(xb, 1.0)
+    np.testing.assert_array_equal(s, rs)
+    np.testing.assert_array_equal(q, rq)
+
+
+@pytest.mark.parametrize("E,N,K", [(3, 32, 128), (2, 40, 2880), (4, 16, 4096)])
+def test_quantize_weights_parity(E, N, K):
+    rng = np.random.default_rng(E * N + K)
+    w = (rng.standard_normal((E, N, K)) * 0.02).astype(np.float32)
+    w[-1] = 0.0 if E > 2 else w[-1]
+    wq = torch.empty((E, N, K // 2), dtype=torch.uint8, device="cuda")
+    sfw = torch.empty((E, N, K // 16), dtype=torch.uint8, device="cuda")
+    gw = torch.empty(E, dtype=torch.float32, device="cuda")
+    moe.moe_quantize_weights_nvfp4(dev(w), E, N, K, wq, sfw, gw)
+    rq, rs, rg = oracle.quantize_weights_nvfp4(w)
+    np.testing.assert_array_equal(gw.cpu().numpy(), rg)
+    np.testing.assert_array_equal(sfw.cpu().numpy(), rs)
+    np.testing.assert_array_equal(wq.cpu().numpy(), rq)
+
+
+# ------------------------------------------------------------------ step 3
+@pytest.mark.parametrize("cfg", [wl.config("tiny"), wl.small_config(K=96, N=9, real=7, E=5, top_k=2),
+                                 wl.config("decode_30b_a3b"),
+                                 wl.small_config(N=300, real=290, K=7168, E=16, top_k=8)])
+def test_dispatch_parity(cfg):
+    x = wl.activations_bf16(cfg)
+    ids = wl.routing(cfg)
+    pipe = RoutingPipeline(cfg.N, cfg.K, cfg.E, cfg.top_k, 64, mode="w4a16")
+    load_inputs(pipe, cfg, x, ids, wl.router_weights(cfg))
+    pipe.recv_buf.fill_(0xA5)
+    pipe.mask()
+    pipe.create_indices()
+    pipe.dispatch_mxfp4()
+    ids_m = oracle.mask_padding(ids, cfg.real)
+    ref_idx = oracle.create_indices(ids_m, cfg.E)
+    check_indices(pipeline_indices(pipe), ref_idx, cfg.slots)
+    ref_recv, ref_counts = oracle.dispatch_mxfp4(x, cfg.top_k, cfg.E, ref_idx, fill=0xA5)
+    np.testing.assert_array_equal(pipe.recv_buf.cpu().numpy(), ref_recv)
+    np.testing.assert_array_equal(host_u32(pipe.recv_counts), ref_counts)
+
+
+def test_dispatch_capacity_overflow_is_reported():
+    cfg = wl.config("tiny")
+    x = wl.activations_bf16(cfg)
+    pipe = RoutingPipeline(cfg.N, cfg.K, cfg.E, cfg.top_k, 64, recv_capacity=10)
+    load_inputs(pipe, cfg, x, wl.routing(cfg), wl.router_weights(cfg))
+    pipe.mask()
+    pipe.create_indices()
+    pipe.dispatch_mxfp4()
+    assert moe.moe_get_device_error(clear=True) & moe.MOE_DEVERR_RECV_OVERFLOW
+    ref_idx = oracle.create_indices(oracle.mask_padding(wl.routing(cfg), cfg.real), cfg.E)
+    ref_recv, _ = oracle.dispatch_mxfp4(x, cfg.top_k, cfg.E, ref_idx)
+    np.testing.assert_array_equal(pipe.recv_buf.cpu().numpy(), ref_recv[:10])
+
+
+# ------------------------------------------------------------------ step 4b
+SENTINEL = 0x4B1D      # bf16 bits of an unlikely finite value (~1.03e7)
+
+GEMV_CASES = [
+    ("tiny-w4a16", wl.config("tiny"), "w4a16"),
+    ("tiny-w4a4", wl.config("tiny"), "w4a4"),
+    # ragged row block (200 % 16 = 8), K % 256 != 0 (4-byte scale copies), 2 chunks
+    ("ragged-w4a16", wl.small_config(), "w4a16"),
+    ("ragged-w4a4", wl.small_config(), "w4a4"),
+    # many tokens per expert: several 32-token passes and full 128-row rounds
+    ("passes-w4a16", wl.small_config("passes", N=300, real=290, K=512, E=4, top_k=2,
+                                     N_out=264), "w4a16"),
+    ("passes-w4a4", wl.small_config("passes", N=300, real=290, K=512, E=4, top_k=2,
+                                    N_out=264), "w4a4"),
+    # minimal K, N
+    ("minimal", wl.small_config("minimal", N=3, real=3, K=64, E=2, top_k=1, N_out=8), "w4a16"),
+    # activations spanning many binades (per-chunk power-of-two scaling)
+    ("wide-range", wl.small_config("wide", N=24, real=24, K=1024, E=6, top_k=2, N_out=128,
+                                   outlier_frac=0.05, outlier_mult=3000.0), "w4a16"),
+]
+
+
+def run_gemv_case(cfg, mode, act_global=1.0):
+    x = wl.activations_bf16(cfg)
+    ids = wl.routing(cfg)
+    pipe = RoutingPipeline(cfg.N, cfg.K, cfg.E, cfg.top_k, cfg.N_out, mode=mode,
+                           act_global=act_global, dispatch=False)
+    load_inputs(pipe, cfg, x, ids, wl.router_weights(cfg))
+    quantize_all_weights(pipe, cfg)
+    pipe.expert_out.view(torch.int16).fill_(SENTINEL)
+    pipe.mask()
+    pipe.create_indices()
+    if mode == "w4a4":
+        pipe.quantize_activations()
+    pipe.gemv()
+    torch.cuda.synchronize()
+    return pipe, x, oracle.mask_padding(ids, cfg.real)
+
+
+@pytest.mark.parametrize("name,cfg,mode", GEMV_CASES, ids=[c[0] for c in GEMV_CASES])
+def test_gemv_parity(name, cfg, mode):
+    g_a = 1.0 if mode == "w4a16" else float(np.float32(0.5))
+    pipe, x, ids = run_gemv_case(cfg, mode, g_a)
+    wq, sfw, gw = oracle_weights(cfg, range(cfg.E))
+    np.testing.assert_array_equal(pipe.wq.cpu().numpy(), wq)
+    np.testing.assert_array_equal(pipe.sfw.cpu().numpy(), sfw)
+    np.testing.assert_array_equal(pipe.w_global.cpu().numpy(), gw)
+    if mode == "w4a16":
+        ref = oracle.grouped_gemv("w4a16", ids, wq, sfw, gw, act_bf16=x)
+    else:
+        xq, sfa = oracle.nvfp4_quantize_bf16(x, g_a)
+        np.testing.assert_array_equal(pipe.xq.cpu().numpy(), xq)
+        np.testing.assert_array_equal(pipe.sfa.cpu().numpy(), sfa)
+        ref = oracle.grouped_gemv("w4a4", ids, wq, sfw, gw, xq=xq, sfa=sfa, g_a=g_a)
+    out_bits = host_bf16_bits(pipe.expert_out)
+    routed = ~np.isnan(ref[..., 0])
+    # unrouted slots are never written
+    assert np.all(out_bits[~routed] == SENTINEL)
+    assert_float_parity(host_bf16_f64(pipe.expert_out)[routed], ref[routed], what=name)
+
+
+def test_gemv_token_major_equals_flattened_pairs():
+    cfg = wl.small_config("flat", N=50, real=44, K=320, E=7, top_k=4, N_out=136)
+    pipe, x, ids = run_gemv_case(cfg, "w4a16")
+    # same pairs as a [R, 1] map: one activation row per (token, slot)
+    R_ids = ids.reshape(-1, 1)
+    xr = np.repeat(x, cfg.top_k, axis=0)
+    flat = RoutingPipeline(cfg.N * cfg.top_k, cfg.K, cfg.E, 1, cfg.N_out, dispatch=False)
+    flat.x.copy_(dev(xr))
+    flat.routing_map.copy_(dev(R_ids))
+    flat.real_token_count.fill_(cfg.N * cfg.top_k)
+    flat.wq.copy_(pipe.wq)
+    flat.sfw.copy_(pipe.sfw)
+    flat.w_global.copy_(pipe.w_global)
+    flat.expert_out.view(torch.int16).fill_(SENTINEL)
+    flat.create_indices()
+    flat.gemv()
+    np.testing.assert_array_equal(host_bf16_bits(flat.expert_out).reshape(-1),
+                                  host_bf16_bits(pipe.expert_out).reshape(-1))
+
+
+def test_gemv_all_slots_unrouted():
+    cfg = wl.small_config("empty", N=8, real=0, K=128, E=4, top_k=2, N_out=32)
+    pipe, x, ids = run_gemv_case(cfg, "w4a16")
+    assert np.all(host_bf16_bits(pipe.expert_out) == SENTINEL)
+    assert host_u32(pipe.expert_usage_stats).tolist() == [0, 0]
+
+
+# ------------------------------------------------------------------ step 5
+@pytest.mark.parametrize("epi,alpha", [("none", 1.0), ("identity", 1.0), ("scale", -0.625)])
+@pytest.mark.parametrize("cfg", [wl.small_config(N=20, real=17, top_k=4, N_out=72, E=6),
+                                 wl.small_config("wide", N=33, real=33, top_k=8, N_out=1000, E=9)])
+def test_combine_parity(cfg, epi, alpha):
+    y = wl.expert_outputs_bf16(cfg)
+    w = wl.router_weights(cfg)
+    ids = oracle.mask_padding(wl.routing(cfg), cfg.real)
+    ids[0, 0] = cfg.E + 3                                   # out of range: routes nowhere
+    out = torch.empty((cfg.N, cfg.N_out), dtype=torch.bfloat16, device="cuda")
+    moe.moe_combine(dev(y), dev(w), dev(ids), cfg.N, cfg.top_k, cfg.N_out, cfg.E,
+                    {"none": 0, "identity": 1, "scale": 2}[epi], alpha, out)
+    ref = oracle.combine(y, w, ids, cfg.E, epi, alpha)
+    assert_float_parity(host_bf16_f64(out), ref, what=f"combine {epi}")
+    assert np.all(host_bf16_f64(out)[cfg.real:] == 0.0)
+
+
+def test_combine_one_hot_is_exact():
+    cfg = wl.small_config(N=8, real=8, top_k=3, N_out=64, E=4)
+    y = wl.expert_outputs_bf16(cfg)
+    ids = np.tile(np.arange(3), (8, 1)).astype(np.int64)
+    w = np.zeros((8, 3), np.float32)
+    sel = np.random.default_rng(2).integers(0, 3, 8)
+    w[np.arange(8), sel] = 1.0
+    out = torch.empty((8, 64), dtype=torch.bfloat16, device="cuda")
+    moe.moe_combine(dev(y), dev(w), dev(ids), 8, 3, 64, cfg.E, 0, 1.0, out)
+    np.testing.assert_array_equal(host_bf16_bits(out), y[np.arange(8), sel])
+
+
+# ------------------------------------------------------------------ boundary
+def test_invalid_arguments_launch_nothing():
+    with pytest.raises(moe.MoeError) as e:
+        moe.moe_grouped_gemv_nvfp4(0, 16, 0, 1.0, 4, 2, 16, 16, 0, 4, 12, 64, 16, 16, 16, 16, 16)
+    assert e.value.status == 1
+    with pytest.raises(moe.MoeError) as e:
+        moe.moe_create_indices(16, 8, 4, 16, 16, 16, 16, 16, None, None, 0)
+    assert e.value.status == 3

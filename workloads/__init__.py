@@ -178,3 +178,18 @@ def all_expert_weights_f32(cfg: Config, experts: Optional[list] = None) -> np.nd
     """Stacked fp32 weights [E, N_out, K] (only for small configs)."""
     es = range(cfg.E) if experts is None else experts
     return np.stack([expert_weights_f32(cfg, e) for e in es])
+
+
+def expert_weights_f32_many(cfg: Config, experts, threads: int = 8) -> np.ndarray:
+    """Stacked fp32 weights of several experts, generated on a thread pool
+    (numpy's generators release the GIL; every expert keeps its own stream)."""
+    from concurrent.futures import ThreadPoolExecutor
+    experts = list(experts)
+    out = np.empty((len(experts), cfg.N_out, cfg.K), np.float32)
+
+    def fill(i):
+        out[i] = expert_weights_f32(cfg, experts[i])
+
+    with ThreadPoolExecutor(max(1, min(threads, len(experts)))) as ex:
+        list(ex.map(fill, range(len(experts))))
+    return out
