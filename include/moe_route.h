@@ -68,6 +68,7 @@ typedef enum {
 /* Bits of the device error word. */
 #define MOE_DEVERR_WAIT_TIMEOUT   0x1u /* a pipeline wait in the GEMV expired           */
 #define MOE_DEVERR_RECV_OVERFLOW  0x2u /* dispatch: routed pairs exceed recv_capacity   */
+#define MOE_DEVERR_ACT_RANGE      0x4u /* W4A16 GEMV: an activation exceeds +-65504     */
 
 /* --------------------------------------------------------------------- */
 /* Step 1 -- Megatron-Core "core.transformer.moe.inference_routing_mask_  */
@@ -183,10 +184,10 @@ MOE_API moe_status_t moe_quantize_weights_nvfp4(const float *w, int32_t E, int32
 /* expert_usage_stats), so "M = routed pairs, top_k = 1" is simply a     */
 /* routing map of shape [R, 1].  w_global may be NULL (all ones).        */
 /* Limits: K % 64 == 0, N % 8 == 0, 1 <= top_k <= E <= 1024; act, w and */
-/* out 16-byte aligned.  W4A16 activations are fed to the tensor cores   */
-/* as fp16 with a per-(token, 256-column chunk) power-of-two scale, so   */
-/* every finite bf16 input is handled; values more than 2^29 below the   */
-/* chunk maximum are rounded to fp16 subnormals.                         */
+/* out 16-byte aligned.  W4A16 activations enter the tensor cores as     */
+/* fp16: exact for 2^-14 <= |x| <= 65504, rounded to fp16 subnormals     */
+/* below (absolute error <= 2^-25); |x| > 65504 raises                   */
+/* MOE_DEVERR_ACT_RANGE (the affected outputs are then undefined).       */
 MOE_API moe_status_t moe_grouped_gemv_nvfp4(moe_gemv_mode_t mode, const void *act, const uint8_t *sfa,
                                     float act_global, int32_t M, int32_t top_k,
                                     const uint8_t *w, const uint8_t *sfw, const float *w_global,

@@ -20,7 +20,7 @@ import threading
 __all__ = [
     "MoeError", "library", "library_path",
     "MOE_W4A16", "MOE_W4A4", "MOE_EPI_NONE", "MOE_EPI_IDENTITY", "MOE_EPI_SCALE",
-    "MOE_DEVERR_WAIT_TIMEOUT", "MOE_DEVERR_RECV_OVERFLOW",
+    "MOE_DEVERR_WAIT_TIMEOUT", "MOE_DEVERR_RECV_OVERFLOW", "MOE_DEVERR_ACT_RANGE",
     "moe_mask_padding", "moe_create_indices_workspace_bytes", "moe_create_indices",
     "moe_mxfp4_row_stride", "moe_dispatch_mxfp4", "moe_quantize_activations_nvfp4",
     "moe_quantize_weights_nvfp4", "moe_grouped_gemv_nvfp4", "moe_combine",
@@ -30,7 +30,7 @@ __all__ = [
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED_ARCH, MOE_ERR_WORKSPACE, MOE_ERR_CUDA = range(5)
 MOE_W4A16, MOE_W4A4 = 0, 1
 MOE_EPI_NONE, MOE_EPI_IDENTITY, MOE_EPI_SCALE = 0, 1, 2
-MOE_DEVERR_WAIT_TIMEOUT, MOE_DEVERR_RECV_OVERFLOW = 0x1, 0x2
+MOE_DEVERR_WAIT_TIMEOUT, MOE_DEVERR_RECV_OVERFLOW, MOE_DEVERR_ACT_RANGE = 0x1, 0x2, 0x4
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_HERE, "libmoe_route.so")

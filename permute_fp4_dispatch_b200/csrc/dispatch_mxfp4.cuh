@@ -6,10 +6,12 @@
 // restore_token_order[p] (from moe_create_indices), so no slot claiming is
 // needed and the row order is deterministic.
 //
-// One warp per token: the row is read once (128-bit loads, 8 bf16 per
-// lane), encoded once, and the encoded 32-bit words are stored to each of
-// the token's routed rows.  A 32-element MX block is 4 lanes; its amax is a
-// 2-step xor-shuffle.  Padding tokens (all slots unrouted) are skipped.
+// One warp per (token, group of up to 8 segments of 256 columns): the row is
+// read once (128-bit loads, 8 bf16 per lane, all of the group's loads in
+// flight together), encoded once, and the encoded 32-bit words are stored to
+// each of the token's routed rows.  A 32-element MX block is 4 lanes; its
+// amax is a 2-step xor-shuffle.  Padding tokens (no routed slot) write
+// nothing.
 #pragma once
 #include "common.cuh"
 
@@ -17,6 +19,7 @@ namespace moe {
 namespace disp {
 
 constexpr int kWarpsPerBlock = 8;
+constexpr int kSegGroup = 8;  // 256-column segments per warp task
 
 // E8M0 exponent of a block: floor(log2(amax)) - 2 clamped to [-127, 127];
 // amax == 0 gives -127.  Exact integer arithmetic on the fp32 bits.
@@ -51,33 +54,46 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     for (uint32_t a = threadIdx.x; a < A; a += blockDim.x)
       counts[expert_ids[a]] = start[a + 1] - start[a];
   }
-  const int warps_total = gridDim.x * kWarpsPerBlock;
+  const int64_t warps_total = (int64_t)gridDim.x * kWarpsPerBlock;
   const int half = K / 2;
   const int nscale = K / 32;
-  for (int t = blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5); t < N; t += warps_total) {
-    // destinations of this token's slots (top_k <= 32 per step)
+  const int segs = (K + 255) / 256;
+  const int groups = (segs + kSegGroup - 1) / kSegGroup;
+  const int64_t tasks = (int64_t)N * groups;
+  for (int64_t task = (int64_t)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5); task < tasks;
+       task += warps_total) {
+    const int t = (int)(task / groups);
+    const int grp = (int)(task % groups);
+    const uint16_t *row = x + (int64_t)t * K;
+    // issue the group's row loads first (independent of the destinations)
+    uint4 v[kSegGroup];
+#pragma unroll
+    for (int q = 0; q < kSegGroup; ++q) {
+      const int k = (grp * kSegGroup + q) * 256 + 8 * (int)lane;
+      v[q] = k < K ? ldg_nc_v4(row + k) : make_uint4(0u, 0u, 0u, 0u);
+    }
     for (int j0 = 0; j0 < top_k; j0 += 32) {
+      // destinations of this token's slots (32 per step)
       const int j = j0 + (int)lane;
       uint32_t dest = 0xFFFFFFFFu;
       if (j < top_k) dest = restore[(int64_t)t * top_k + j];
       bool ok = dest != 0xFFFFFFFFu;
       if (ok && (int64_t)dest >= capacity) {
-        raise_device_error(MOE_DEVERR_RECV_OVERFLOW);
+        if (grp == 0) raise_device_error(MOE_DEVERR_RECV_OVERFLOW);
         ok = false;
       }
       const unsigned dmask = __ballot_sync(0xffffffffu, ok);
       if (dmask == 0u) continue;
-      const uint16_t *row = x + (int64_t)t * K;
-      for (int seg = 0; seg < K; seg += 256) {
-        const int k = seg + 8 * (int)lane;
+#pragma unroll
+      for (int q = 0; q < kSegGroup; ++q) {
+        const int k = (grp * kSegGroup + q) * 256 + 8 * (int)lane;
+        if ((grp * kSegGroup + q) * 256 >= K) break;  // warp-uniform
         const bool active = k < K;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (active) v = ldg_nc_v4(row + k);
         float f[8];
-        f[0] = bf16_lo(v.x); f[1] = bf16_hi(v.x);
-        f[2] = bf16_lo(v.y); f[3] = bf16_hi(v.y);
-        f[4] = bf16_lo(v.z); f[5] = bf16_hi(v.z);
-        f[6] = bf16_lo(v.w); f[7] = bf16_hi(v.w);
+        f[0] = bf16_lo(v[q].x); f[1] = bf16_hi(v[q].x);
+        f[2] = bf16_lo(v[q].y); f[3] = bf16_hi(v[q].y);
+        f[4] = bf16_lo(v[q].z); f[5] = bf16_hi(v[q].z);
+        f[6] = bf16_lo(v[q].w); f[7] = bf16_hi(v[q].w);
         float amax = 0.0f;
 #pragma unroll
         for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
@@ -85,10 +101,10 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
         amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
         const int se = mx_shared_exponent(amax);
         const float mult = __uint_as_float((uint32_t)(127 - se) << 23);  // 2^-se, exact
-        float q[8];
+        float qv[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) q[i] = f[i] * mult;
-        const uint32_t codes = e2m1x8_from_f32(q);
+        for (int i = 0; i < 8; ++i) qv[i] = f[i] * mult;
+        const uint32_t codes = e2m1x8_from_f32(qv);
         // store to every routed row of this token
         unsigned m = dmask;
         while (m) {
@@ -102,14 +118,16 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
           }
         }
       }
-      // zero padding after the scales
-      const int pad0 = half + nscale;
-      unsigned m = dmask;
-      while (m) {
-        const int src = __ffs(m) - 1;
-        m &= m - 1;
-        const uint32_t d = __shfl_sync(0xffffffffu, dest, src);
-        for (int b = pad0 + (int)lane; b < stride; b += 32) recv[(int64_t)d * stride + b] = 0;
+      // zero padding after the scales (written by the group that holds the last segment)
+      if (grp == groups - 1) {
+        const int pad0 = half + nscale;
+        unsigned m = dmask;
+        while (m) {
+          const int src = __ffs(m) - 1;
+          m &= m - 1;
+          const uint32_t d = __shfl_sync(0xffffffffu, dest, src);
+          for (int b = pad0 + (int)lane; b < stride; b += 32) recv[(int64_t)d * stride + b] = 0;
+        }
       }
     }
   }

@@ -6,63 +6,77 @@
 // [M, top_k, N]).  For each routed pair p with expert e:
 //     out[p, n] = bf16( g_w[e] * g_a * sum_k a(p/top_k, k) * w(e, n, k) ).
 //
-// Design (decode-first, HBM-bound on the weight stream):
-//   * Work is expert-major: the pairs of an active expert (CSR from
-//     moe_create_indices) are processed in passes of up to kTS = 32 tokens,
-//     and each pass sweeps the expert's N rows in 16-row blocks.  The flat
-//     list of (expert, pass, row block) units is split into equal contiguous
-//     ranges, one per persistent CTA (grid = SM count), so the weight bytes
-//     per CTA are balanced to one 16-row block.
-//   * A CTA = 1 producer warp + 8 consumer warps.  Consecutive blocks of one
-//     (expert, pass) form a round of up to 128 rows.  The producer streams
-//     each round's FP4 rows and E4M3 scales in chunks of kKC = 256 columns
-//     into a 4-stage shared-memory ring with bulk copies on the TMA engine
-//     (cp.async.bulk, mbarrier transaction counts); scale rows that are not
-//     16-byte aligned use 4-byte cp.async instead.
-//   * Consumers dequantise in registers, exactly: E2M1 -> f16x2 with the
-//     hardware converter, times the block's E4M3 scale (a product of at most
-//     6 significant bits, exact in fp16), and feed warp-level tensor-core MMAs
-//     (m16n8k16, fp32 accumulation) with the tokens on the n = 8 side.
-//     Within a 64-column span each lane owns 16 contiguous columns (one scale
-//     block); A and B use the same column permutation, so the dot product is
-//     unchanged.
-//   * Activations are staged per chunk by the consumers themselves into a
-//     double-buffered fp16 tile laid out in fragment order with an XOR
-//     swizzle (conflict-free 128-bit loads and stores).  W4A16 rows are scaled
-//     by a per-(token, chunk) power of two so the chunk maximum lies in
-//     [2^14, 2^15) before the fp16 conversion (exact for every value within
-//     2^29 of the chunk maximum); the power of two is undone in fp32 after
-//     the chunk.  W4A4 activations are dequantised exactly like the weights.
-//   * The round's accumulators are scaled by g_w * g_a, rounded to bf16,
-//     transposed through shared memory and written as 16-byte row segments.
+// Design (decode-first; the FP4 weight stream is the roofline):
+//   * Work is expert-major: an active expert's pairs (CSR from
+//     moe_create_indices) are taken in passes of up to kTS = 64 tokens and
+//     each pass sweeps the expert's N rows in 16-row blocks.  The flat list of
+//     (expert, pass, row block) units is split into equal contiguous ranges,
+//     one per persistent CTA (grid = SM count).  Consecutive blocks of one
+//     (expert, pass) form a round of up to 128 rows: one tcgen05 MMA tile
+//     (M = 128 weight rows, N = tokens rounded up to 16, fp32 in TMEM).
+//   * Warp roles (10 warps):
+//       warp 8      TMA producer: streams each round's FP4 rows and E4M3
+//                   scales in chunks of kKC = 256 columns into a kStages-deep
+//                   shared-memory ring (one 16-row x 128-byte box per row
+//                   block, 128-byte swizzle, L2 evict-first; rows past N and
+//                   columns past K arrive as zeros; scale rows whose stride is
+//                   not a multiple of 16 bytes use 4-byte cp.async);
+//       warps 0-7   dequantise: each lane owns one weight row (warp w covers
+//                   TMEM lanes 32*(w%4).. and columns half w/4 of the chunk),
+//                   E2M1 -> f16x2 with the hardware converter, times the
+//                   block's E4M3 scale (at most 6 significant bits: exact in
+//                   fp16), written to a double-buffered A tile in tensor
+//                   memory with tcgen05.st; they also stage the chunk's
+//                   activations as fp16 into a double-buffered, 128B-swizzled
+//                   K-major B tile, and run the output epilogue;
+//       warp 9      allocates TMEM and issues tcgen05.mma kind::f16 (A from
+//                   TMEM, B from shared memory) for every chunk, committing to
+//                   mbarriers that free the A/B buffers and publish D.
+//     D is double-buffered in TMEM, so a round's epilogue (tcgen05.ld, scale
+//     by g_w * g_a, round to bf16, store) runs while the next round's first
+//     chunk is already being multiplied.
+//   * W4A16 activations enter the tensor core as fp16: exact for
+//     2^-14 <= |x| <= 65504, fp16-subnormal rounding (absolute error
+//     <= 2^-25) below; |x| > 65504 raises MOE_DEVERR_ACT_RANGE.  W4A4
+//     activations are dequantised exactly like the weights.
 #pragma once
 #include "common.cuh"
 
 namespace moe {
 namespace gemv {
 
-constexpr int kCW = 8;                  // consumer warps
-constexpr int kThreads = (kCW + 1) * 32;
-constexpr int kRows = 16 * kCW;         // rows per round
+constexpr int kDQ = 8;                  // dequant / staging / epilogue warps
+constexpr int kTmaWarp = kDQ;
+constexpr int kMmaWarp = kDQ + 1;
+constexpr int kThreads = (kDQ + 2) * 32;
+constexpr int kBlocksPerRound = 8;      // 16-row blocks per round (M = 128)
 constexpr int kKC = 256;                // columns (codes) per chunk
-constexpr int kTS = 32;                 // tokens per pass
-constexpr int kNG = kTS / 8;            // n8 groups per pass
-constexpr int kStages = 4;
-constexpr int kWStride = kKC / 2 + 16;  // bytes per weight row in a stage (padded)
+constexpr int kTS = 64;                 // tokens per pass (MMA N <= 64)
+constexpr int kStages = 5;
+constexpr int kWStride = kKC / 2;       // bytes per weight row in a stage (128B-swizzled)
 constexpr int kSFStride = kKC / 16;     // bytes per scale row in a stage
-constexpr int kStageW = kRows * kWStride;
-constexpr int kStageBytes = kStageW + kRows * kSFStride;
-constexpr int kActBytes = kTS * kKC * 2;
-constexpr int kStagingBytes = kCW * kTS * 16 * 2;
+constexpr int kBoxW = 16 * kWStride;    // one 16-row weight box
+constexpr int kBoxSF = 16 * kSFStride;  // one 16-row scale box
+constexpr int kStageW = 128 * kWStride;
+constexpr int kStageBytes = kStageW + 128 * kSFStride;
+constexpr int kKatomBytes = kTS * 128;  // one 64-column slab of the B tile
+constexpr int kBTile = 4 * kKatomBytes;
 constexpr int kMaxExperts = 1024;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kAcol = 0;           // A tiles: columns [0, 256), 128 per buffer
+constexpr uint32_t kDcol = 256;         // D tiles: columns [256, 384), 64 per buffer
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
-constexpr size_t kOffAct = (size_t)kStages * kStageBytes;
-constexpr size_t kOffCS = kOffAct + 2 * kActBytes;
-constexpr size_t kOffStaging = kOffCS + 2 * kTS * 4;
-constexpr size_t kOffPrefix = kOffStaging + kStagingBytes;
-constexpr size_t kOffBar = kOffPrefix + (kMaxExperts + 4) * 4;
-constexpr size_t kSmemBytes = kOffBar + 2 * kStages * 8 + 16;
+static_assert(kStageBytes % 1024 == 0, "stages must keep the 1024-byte swizzle alignment");
+constexpr size_t kOffB = (size_t)kStages * kStageBytes;
+constexpr size_t kOffPrefix = kOffB + 2 * kBTile;
+constexpr size_t kOffStart = kOffPrefix + (kMaxExperts + 4) * 4;
+constexpr size_t kOffEid = kOffStart + (kMaxExperts + 4) * 4;
+constexpr size_t kOffPair = kOffEid + (kMaxExperts + 4) * 4;     // [2][kTS] pair ids
+constexpr size_t kOffBar = kOffPair + 2 * kTS * 4;
+constexpr int kNumBars = 2 * kStages + 8;
+constexpr size_t kOffMisc = kOffBar + kNumBars * 8;             // tmem slot, abort flag
+constexpr size_t kSmemBytes = kOffMisc + 16 + 1024;             // + alignment slack
 
 struct Params {
   const void *act;          // W4A16: bf16 [M, K]; W4A4: u8 [M, K/2]
@@ -89,48 +103,63 @@ struct Round {
   int nblk;
 };
 
-// Next round of this CTA's unit range; identical in every warp.
-__device__ __forceinline__ bool next_round(uint32_t &u, uint32_t u_end, int &a,
-                                           const uint32_t *prefix, const Params &p, int RB,
-                                           Round &r) {
-  if (u >= u_end) return false;
-  while (u >= prefix[a + 1]) ++a;
-  const uint32_t v = u - prefix[a];
-  const uint32_t pass = v / (uint32_t)RB;
-  const uint32_t rb = v % (uint32_t)RB;
-  uint32_t nblk = (uint32_t)RB - rb;
-  if (nblk > (uint32_t)kCW) nblk = kCW;
-  if (nblk > u_end - u) nblk = u_end - u;
-  const uint32_t s0 = p.start[a];
-  const uint32_t c = p.start[a + 1] - s0;
-  r.e = p.eids[a];
-  r.tok0 = s0 + pass * kTS;
-  r.ntok = (int)min((uint32_t)kTS, c - pass * kTS);
-  r.n0 = (int)rb * 16;
-  r.nrows = min((int)nblk * 16, p.N - r.n0);
-  r.nblk = (int)nblk;
-  u += nblk;
-  return true;
-}
+// Per-expert metadata staged in shared memory at kernel start.
+struct Meta {
+  const uint32_t *prefix;  // units before active expert a
+  const uint32_t *start;   // CSR offsets
+  const int32_t *eid;      // expert ids
+  int N;
+};
+
+// Walks a CTA's unit range round by round; identical in every thread.
+struct RoundIter {
+  uint32_t u, u_end;
+  int a;
+  __device__ __forceinline__ bool next(const Meta &m, int RB, Round &r) {
+    if (u >= u_end) return false;
+    while (u >= m.prefix[a + 1]) ++a;
+    const uint32_t v = u - m.prefix[a];
+    const uint32_t pass = v / (uint32_t)RB;
+    const uint32_t rb = v % (uint32_t)RB;
+    uint32_t nblk = (uint32_t)RB - rb;
+    if (nblk > (uint32_t)kBlocksPerRound) nblk = kBlocksPerRound;
+    if (nblk > u_end - u) nblk = u_end - u;
+    const uint32_t s0 = m.start[a];
+    const uint32_t c = m.start[a + 1] - s0;
+    r.e = m.eid[a];
+    r.tok0 = s0 + pass * kTS;
+    r.ntok = (int)min((uint32_t)kTS, c - pass * kTS);
+    r.n0 = (int)rb * 16;
+    r.nrows = min((int)nblk * 16, m.N - r.n0);
+    r.nblk = (int)nblk;
+    u += nblk;
+    return true;
+  }
+};
 
 __device__ __forceinline__ uint32_t bcast_lo(uint32_t h) { return __byte_perm(h, h, 0x1010); }
 __device__ __forceinline__ uint32_t bcast_hi(uint32_t h) { return __byte_perm(h, h, 0x3232); }
 
-// fp16 tile index (in 16-byte units) of (group G, span s, half h, lane (g,t)).
-__device__ __forceinline__ int act_chunk16(int G, int s, int h, int g, int t) {
-  return ((G * 4 + s) * 2 + h) * 32 + ((g * 4 + t) ^ (2 * s + h));
-}
-
-template <int MODE, bool SF_BULK>
-__global__ void __launch_bounds__(kThreads, 1) grouped_gemv_kernel(const Params p) {
-  extern __shared__ __align__(1024) uint8_t smem[];
-  uint8_t *act_tile = smem + kOffAct;
-  float *cs_tile = reinterpret_cast<float *>(smem + kOffCS);
-  uint16_t *staging = reinterpret_cast<uint16_t *>(smem + kOffStaging);
+template <int MODE, bool SF_TMA>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_gemv_kernel(const Params p, const __grid_constant__ CUtensorMap tmap_w,
+                        const __grid_constant__ CUtensorMap tmap_sf) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t *btile = smem + kOffB;
   uint32_t *prefix = reinterpret_cast<uint32_t *>(smem + kOffPrefix);
+  uint32_t *s_start = reinterpret_cast<uint32_t *>(smem + kOffStart);
+  int32_t *s_eid = reinterpret_cast<int32_t *>(smem + kOffEid);
+  uint32_t *s_pair = reinterpret_cast<uint32_t *>(smem + kOffPair);
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + kOffBar);
   uint64_t *empty = full + kStages;
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(empty + kStages);
+  uint64_t *a_full = empty + kStages;   // [2]
+  uint64_t *a_empty = a_full + 2;       // [2]
+  uint64_t *d_full = a_empty + 2;       // [2]
+  uint64_t *d_empty = d_full + 2;       // [2]
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffMisc);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffMisc + 8);
 
   const int warp = threadIdx.x >> 5;
   const int lane = (int)lane_id();
@@ -159,263 +188,322 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemv_kernel(const Params 
     }
     if (lane == 0) prefix[0] = 0;
   }
+  for (uint32_t i = threadIdx.x; i <= A; i += blockDim.x) {
+    s_start[i] = p.start[i];
+    if (i < A) s_eid[i] = p.eids[i];
+  }
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full[s], SF_BULK ? 1u : 33u);
-      mbar_init(&empty[s], (uint32_t)kCW);
+      mbar_init(&full[s], SF_TMA ? 1u : 33u);
+      mbar_init(&empty[s], (uint32_t)kDQ);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&a_full[b], (uint32_t)kDQ);
+      mbar_init(&a_empty[b], 1u);
+      mbar_init(&d_full[b], 1u);
+      mbar_init(&d_empty[b], (uint32_t)kDQ);
     }
     *abort_flag = 0;
     fence_mbar_init();
   }
+  if (warp == kMmaWarp) tmem_alloc(tmem_slot, kTmemCols);
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
 
   const uint32_t U = prefix[A];
   const uint32_t u_begin = (uint32_t)(((uint64_t)U * blockIdx.x) / gridDim.x);
   const uint32_t u_end = (uint32_t)(((uint64_t)U * (blockIdx.x + 1)) / gridDim.x);
   const int nchunks = (K + kKC - 1) / kKC;
-  const int64_t row_bytes = K / 2, sf_row_bytes = K / 16;
+  const int64_t sf_row_bytes = K / 16;
+  const Meta meta{prefix, s_start, s_eid, N};
 
-  if (warp == kCW) {
-    // ---------------------------------------------------------------- producer
-    uint32_t u = u_begin, it = 0;
-    int a = 0;
+  auto wait = [&](uint64_t *bar, uint32_t parity) {
+    if (*abort_flag) return;
+    if (!mbar_wait_bounded(bar, parity, kWaitLimitNs)) *abort_flag = 1;
+  };
+
+  if (warp == kTmaWarp) {
+    // ================================================================ TMA producer
+    RoundIter iter{u_begin, u_end, 0};
     Round r;
-    while (next_round(u, u_end, a, prefix, p, RB, r)) {
-      const uint8_t *wbase = p.w + ((int64_t)r.e * N + r.n0) * row_bytes;
-      const uint8_t *sbase = p.sfw + ((int64_t)r.e * N + r.n0) * sf_row_bytes;
+    uint32_t it = 0;
+    const uint64_t policy = l2_evict_first_policy();
+    if (lane == 0) {
+      prefetch_tmap(&tmap_w);
+      if (SF_TMA) prefetch_tmap(&tmap_sf);
+    }
+    while (iter.next(meta, RB, r)) {
       for (int c = 0; c < nchunks; ++c, ++it) {
         const int s = (int)(it % kStages);
-        const uint32_t ph = (it / kStages) & 1u;
-        if (!*abort_flag && !mbar_wait_bounded(&empty[s], ph ^ 1u, kWaitLimitNs)) *abort_flag = 1;
+        wait(&empty[s], ((it / kStages) & 1u) ^ 1u);
         if (*abort_flag) continue;
         const int k0 = c * kKC;
-        const int kcb = min(kKC, K - k0);
-        const uint32_t wb = (uint32_t)kcb / 2, sb = (uint32_t)kcb / 16;
         uint8_t *sw = smem + (size_t)s * kStageBytes;
         uint8_t *ssf = sw + kStageW;
         if (lane == 0)
-          mbar_arrive_expect_tx(&full[s], (uint32_t)r.nrows * (wb + (SF_BULK ? sb : 0u)));
-        for (int row = lane; row < r.nrows; row += 32) {
-          bulk_g2s(sw + row * kWStride, wbase + row * row_bytes + k0 / 2, wb, &full[s]);
-          const uint8_t *src = sbase + row * sf_row_bytes + k0 / 16;
-          if (SF_BULK) {
-            bulk_g2s(ssf + row * kSFStride, src, sb, &full[s]);
-          } else {
-            for (uint32_t q = 0; q < sb; q += 4) cp_async4(ssf + row * kSFStride + q, src + q);
-          }
+          mbar_arrive_expect_tx(&full[s], (uint32_t)r.nblk * (kBoxW + (SF_TMA ? kBoxSF : 0)));
+        __syncwarp();
+        if (lane < r.nblk) {
+          tma_load_3d(sw + lane * kBoxW, &tmap_w, k0 / 2, r.n0 + 16 * lane, r.e, &full[s], policy);
+          if (SF_TMA)
+            tma_load_3d(ssf + lane * kBoxSF, &tmap_sf, k0 / 16, r.n0 + 16 * lane, r.e, &full[s],
+                        policy);
         }
-        if (!SF_BULK) cp_async_mbar_arrive_noinc(&full[s]);
+        if (!SF_TMA) {
+          const uint32_t sb = (uint32_t)min(kKC, K - k0) / 16;
+          const uint8_t *sbase = p.sfw + ((int64_t)r.e * N + r.n0) * sf_row_bytes + k0 / 16;
+          for (int row = lane; row < r.nrows; row += 32)
+            for (uint32_t q = 0; q < sb; q += 4)
+              cp_async4(ssf + row * kSFStride + q, sbase + row * sf_row_bytes + q);
+          cp_async_mbar_arrive_noinc(&full[s]);
+        }
       }
     }
-    return;
-  }
-
-  // ------------------------------------------------------------------ consumers
-  const int cw = warp;
-  const int g = lane >> 2, t = lane & 3;
-  // converter lane mapping: lane L owns chunk columns [8L, 8L+8)
-  const int cv_t = lane >> 3, cv_s = (lane & 7) >> 1, cv_h = lane & 1;
-  uint32_t u = u_begin, it = 0;
-  int a = 0;
-  Round r;
-  while (next_round(u, u_end, a, prefix, p, RB, r)) {
-    const int ngroups = (r.ntok + 7) / 8;
-    // rows of the tokens this warp converts: tau = cw + 8 i
-    int64_t arow[kNG];
-    bool tv[kNG];
-#pragma unroll
-    for (int i = 0; i < kNG; ++i) {
-      const int tau = cw + 8 * i;
-      tv[i] = tau < r.ntok;
-      arow[i] = tv[i] ? (int64_t)(p.order[r.tok0 + tau] / (uint32_t)p.top_k) : 0;
+  } else if (warp == kMmaWarp) {
+    // ================================================================ MMA issuer
+    if (lane == 0) {
+      RoundIter iter{u_begin, u_end, 0};
+      Round r;
+      uint32_t it = 0, rnd = 0;
+      while (iter.next(meta, RB, r)) {
+        const uint32_t d = rnd & 1u;
+        wait(&d_empty[d], ((rnd >> 1) & 1u) ^ 1u);
+        tc_fence_after();
+        const int nmma = (r.ntok + 15) / 16 * 16;
+        const uint32_t idesc = umma_idesc_f16(128, nmma);
+        const uint32_t d_t = tbase + kDcol + d * 64u;
+        for (int c = 0; c < nchunks; ++c, ++it) {
+          const uint32_t b = it & 1u;
+          wait(&a_full[b], (it >> 1) & 1u);
+          tc_fence_after();
+          const int ksteps = min(kKC, K - c * kKC) / 16;
+          if (!*abort_flag) {
+            const uint32_t bbase = smem_addr(btile + b * kBTile);
+            for (int j = 0; j < ksteps; ++j) {
+              const uint64_t bdesc =
+                  umma_desc_sw128(bbase + (uint32_t)(j >> 2) * kKatomBytes + (uint32_t)(j & 3) * 32u,
+                                  1024u);
+              umma_f16_ts(d_t, tbase + kAcol + b * 128u + 8u * (uint32_t)j, bdesc, idesc,
+                          (c > 0 || j > 0) ? 1u : 0u);
+            }
+          }
+          umma_commit(&a_empty[b]);
+        }
+        umma_commit(&d_full[d]);
+        ++rnd;
+      }
     }
-    // prefetch chunk 0 of the activations
-    uint4 raw[kNG];
-    auto load_act = [&](int c) {
+    __syncwarp();
+  } else {
+    // ================================================================ dequant / staging / epilogue
+    const int q = warp & 3;     // TMEM lane quarter
+    const int h = warp >> 2;    // column half of a chunk
+    const int row = 32 * q + lane;
+    const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+    RoundIter iter{u_begin, u_end, 0};
+    Round r, rn, rp;  // current, next, previous (pending epilogue)
+    bool have = iter.next(meta, RB, r);
+    bool have_n = have && iter.next(meta, RB, rn);
+    bool ep_pending = false;
+    uint32_t it = 0, rnd = 0, rnd_p = 0;
+    // token pair ids of the current / next round, one token per lane (lanes < 8):
+    // lane i of warp w holds token tau = w + 8 i
+    uint32_t pair_cur = 0xFFFFFFFFu, pair_nxt = 0xFFFFFFFFu;
+    auto fetch_pairs = [&](const Round &q_, uint32_t &dst) {
+      const int tau = warp + 8 * lane;
+      dst = (lane < 8 && tau < q_.ntok) ? p.order[q_.tok0 + tau] : 0xFFFFFFFFu;
+    };
+    if (have) fetch_pairs(r, pair_cur);
+
+    // activations of this warp's tokens for one chunk (8 values per lane per token)
+    uint4 raw[8];
+    auto load_act = [&](uint32_t pairs, int ntok, int c) {
       const int k0 = c * kKC;
       const int kcb = min(kKC, K - k0);
       const bool kv = 8 * lane < kcb;
 #pragma unroll
-      for (int i = 0; i < kNG; ++i) {
+      for (int i = 0; i < 8; ++i) {
         raw[i] = make_uint4(0u, 0u, 0u, 0u);
-        if (tv[i] && kv) {
+        const uint32_t pr = __shfl_sync(0xffffffffu, pairs, i);
+        if (warp + 8 * i < ntok && kv) {
+          const int64_t m = (int64_t)(pr / (uint32_t)p.top_k);
           if (MODE == MOE_W4A16) {
-            raw[i] = ldg_nc_v4(static_cast<const uint16_t *>(p.act) + arow[i] * K + k0 + 8 * lane);
+            raw[i] = ldg_nc_v4(static_cast<const uint16_t *>(p.act) + m * K + k0 + 8 * lane);
           } else {
-            const uint8_t *q = static_cast<const uint8_t *>(p.act) + arow[i] * (K / 2);
-            raw[i].x = __ldg(reinterpret_cast<const uint32_t *>(q + (k0 + 8 * lane) / 2));
-            raw[i].y = p.sfa[arow[i] * (K / 16) + (k0 + 8 * lane) / 16];
+            const uint8_t *qp = static_cast<const uint8_t *>(p.act) + m * (K / 2);
+            raw[i].x = __ldg(reinterpret_cast<const uint32_t *>(qp + (k0 + 8 * lane) / 2));
+            raw[i].y = p.sfa[m * (K / 16) + (k0 + 8 * lane) / 16];
           }
         }
       }
     };
-    load_act(0);
+    if (have) load_act(pair_cur, r.ntok, 0);
 
-    float acc[kNG][4];
+    auto epilogue = [&](const Round &er, uint32_t ernd) {
+      const uint32_t d = ernd & 1u;
+      wait(&d_full[d], (ernd >> 1) & 1u);
+      tc_fence_after();
+      const int c0 = 32 * h;  // this warp's token columns
+      uint32_t v[32];
+      const bool cols = c0 < er.ntok && 32 * q < er.nrows;
+      if (cols) {
+        uint32_t t0[16], t1[16];
+        const uint32_t ta = tbase + lane_base + kDcol + d * 64u + (uint32_t)c0;
+        tmem_ld16(ta, t0);
+        tmem_ld16(ta + 16u, t1);
+        tmem_wait_ld();
 #pragma unroll
-    for (int G = 0; G < kNG; ++G)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) acc[G][i] = 0.f;
-
-    const bool has_rows = cw < r.nblk;
-    const int wrow = cw * 16 + g;  // row of a0 within the round (row + 8 for a1)
-
-    for (int c = 0; c < nchunks; ++c, ++it) {
-      const int buf = (int)(it & 1u);
-      const int k0 = c * kKC;
-      const int kcb = min(kKC, K - k0);
-      uint4 *tile = reinterpret_cast<uint4 *>(act_tile + buf * kActBytes);
-      float *cs = cs_tile + buf * kTS;
-      // ---- convert this chunk's activations into the fp16 fragment tile
-#pragma unroll
-      for (int i = 0; i < kNG; ++i) {
-        if (!tv[i]) continue;  // warp-uniform
-        uint4 h;
-        float back = 1.0f;
-        if (MODE == MOE_W4A16) {
-          float f[8];
-          f[0] = bf16_lo(raw[i].x); f[1] = bf16_hi(raw[i].x);
-          f[2] = bf16_lo(raw[i].y); f[3] = bf16_hi(raw[i].y);
-          f[4] = bf16_lo(raw[i].z); f[5] = bf16_hi(raw[i].z);
-          f[6] = bf16_lo(raw[i].w); f[7] = bf16_hi(raw[i].w);
-          float m = 0.f;
-#pragma unroll
-          for (int q = 0; q < 8; ++q) m = fmaxf(m, fabsf(f[q]));
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-          float inv = 1.0f;
-          if (m > 0.f) {
-            const int ex = (int)((__float_as_uint(m) >> 23) & 0xFFu);
-            int sig = ex - 141;  // floor(log2 m) - 14 for normal m
-            sig = sig < -126 ? -126 : sig;
-            inv = __uint_as_float((uint32_t)(127 - sig) << 23);
-            back = __uint_as_float((uint32_t)(127 + sig) << 23);
-          }
-          h.x = pack_f16x2(f[0] * inv, f[1] * inv);
-          h.y = pack_f16x2(f[2] * inv, f[3] * inv);
-          h.z = pack_f16x2(f[4] * inv, f[5] * inv);
-          h.w = pack_f16x2(f[6] * inv, f[7] * inv);
-        } else {
-          uint32_t q0, q1, q2, q3;
-          e2m1x8_to_f16x2(raw[i].x, q0, q1, q2, q3);
-          const uint32_t sc = bcast_lo(e4m3x2_to_f16x2(raw[i].y));
-          h.x = hmul2(q0, sc);
-          h.y = hmul2(q1, sc);
-          h.z = hmul2(q2, sc);
-          h.w = hmul2(q3, sc);
+        for (int i = 0; i < 16; ++i) {
+          v[i] = t0[i];
+          v[16 + i] = t1[i];
         }
-        tile[act_chunk16(i, cv_s, cv_h, cw, cv_t)] = h;
-        if (lane == 0) cs[cw + 8 * i] = back;
       }
-      named_bar_sync(1, kCW * 32);
-      if (c + 1 < nchunks) load_act(c + 1);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&d_empty[d]);
+      if (cols && !*abort_flag && row < er.nrows) {
+        const float gw = p.w_global ? p.w_global[er.e] : 1.0f;
+        const float f = __fmul_rn(gw, p.g_a);
+        const int n = er.n0 + row;
+        const uint32_t *pairs = s_pair + (ernd & 1u) * kTS;
+        const int ncol = min(32, er.ntok - c0);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          if (i < ncol) {
+            const uint32_t pr = pairs[c0 + i];
+            const __nv_bfloat16 o = __float2bfloat16_rn(__uint_as_float(v[i]) * f);
+            p.out[(int64_t)pr * N + n] = __bfloat16_as_ushort(o);
+          }
+        }
+      }
+    };
 
-      const int s = (int)(it % kStages);
-      const uint32_t ph = (it / kStages) & 1u;
-      if (!*abort_flag && !mbar_wait_bounded(&full[s], ph, kWaitLimitNs)) *abort_flag = 1;
+    while (have) {
+      // ---- round start: publish this round's pair ids, fetch the next round's
+      named_bar_sync(1, kDQ * 32);
+      if (lane < 8 && warp + 8 * lane < r.ntok)
+        s_pair[(rnd & 1u) * kTS + warp + 8 * lane] = pair_cur;
+      if (have_n) fetch_pairs(rn, pair_nxt);
+      named_bar_sync(1, kDQ * 32);
+      const bool has_rows = 32 * q < r.nrows;
 
-      if (!*abort_flag && has_rows) {
+      for (int c = 0; c < nchunks; ++c, ++it) {
+        const int s = (int)(it % kStages);
+        const uint32_t b = it & 1u;
+        const int k0 = c * kKC;
+        const int kcb = min(kKC, K - k0);
+        // ---- weights of this chunk: this lane's row, columns [128h, 128h + 128)
+        wait(&full[s], (it / kStages) & 1u);
         const uint8_t *sw = smem + (size_t)s * kStageBytes;
         const uint8_t *ssf = sw + kStageW;
-        const bool lane_k = 64 * t < kcb;
-        uint4 wa[2], wb[2];
-        uint32_t sfa_w = 0, sfb_w = 0;
-        if (lane_k) {
-          const uint4 *pa = reinterpret_cast<const uint4 *>(sw + wrow * kWStride + 32 * t);
-          const uint4 *pb = reinterpret_cast<const uint4 *>(sw + (wrow + 8) * kWStride + 32 * t);
-          wa[0] = pa[0]; wa[1] = pa[1];
-          wb[0] = pb[0]; wb[1] = pb[1];
-          sfa_w = *reinterpret_cast<const uint32_t *>(ssf + wrow * kSFStride + 4 * t);
-          sfb_w = *reinterpret_cast<const uint32_t *>(ssf + (wrow + 8) * kSFStride + 4 * t);
-        } else {
-          wa[0] = wa[1] = wb[0] = wb[1] = make_uint4(0u, 0u, 0u, 0u);
-        }
-        const uint32_t sa01 = e4m3x2_to_f16x2(sfa_w & 0xFFFFu), sa23 = e4m3x2_to_f16x2(sfa_w >> 16);
-        const uint32_t sb01 = e4m3x2_to_f16x2(sfb_w & 0xFFFFu), sb23 = e4m3x2_to_f16x2(sfb_w >> 16);
-        float d[kNG][4];
+        uint4 wv[4];
+        uint2 sv = make_uint2(0u, 0u);
+        if (has_rows) {
 #pragma unroll
-        for (int G = 0; G < kNG; ++G)
-#pragma unroll
-          for (int i = 0; i < 4; ++i) d[G][i] = 0.f;
-#pragma unroll
-        for (int sp = 0; sp < 4; ++sp) {
-          const uint32_t sca = (sp & 1) ? bcast_hi(sp < 2 ? sa01 : sa23) : bcast_lo(sp < 2 ? sa01 : sa23);
-          const uint32_t scb = (sp & 1) ? bcast_hi(sp < 2 ? sb01 : sb23) : bcast_lo(sp < 2 ? sb01 : sb23);
-          const uint4 &va = wa[sp >> 1];
-          const uint4 &vb = wb[sp >> 1];
-          const uint32_t ca0 = (sp & 1) ? va.z : va.x, ca1 = (sp & 1) ? va.w : va.y;
-          const uint32_t cb0 = (sp & 1) ? vb.z : vb.x, cb1 = (sp & 1) ? vb.w : vb.y;
-          uint32_t A0[4], A1[4], B0[4], B1[4];
-          e2m1x8_to_f16x2(ca0, A0[0], A0[1], A0[2], A0[3]);  // row g, MMAs 0,1
-          e2m1x8_to_f16x2(ca1, A1[0], A1[1], A1[2], A1[3]);  // row g, MMAs 2,3
-          e2m1x8_to_f16x2(cb0, B0[0], B0[1], B0[2], B0[3]);  // row g+8
-          e2m1x8_to_f16x2(cb1, B1[0], B1[1], B1[2], B1[3]);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            A0[q] = hmul2(A0[q], sca);
-            A1[q] = hmul2(A1[q], sca);
-            B0[q] = hmul2(B0[q], scb);
-            B1[q] = hmul2(B1[q], scb);
+          for (int jj = 0; jj < 4; ++jj) {
+            const int ci = 4 * h + jj;  // logical 16-byte chunk of the 128-byte row
+            wv[jj] = (128 * h + 32 * jj < kcb)
+                         ? *reinterpret_cast<const uint4 *>(sw + row * kWStride + ((ci ^ (row & 7)) * 16))
+                         : make_uint4(0u, 0u, 0u, 0u);
           }
+          sv = *reinterpret_cast<const uint2 *>(ssf + row * kSFStride + 8 * h);
+        }
+        // ---- A/B buffer b is free once the MMAs of item it - 2 completed
+        wait(&a_empty[b], ((it >> 1) & 1u) ^ 1u);
+        tc_fence_after();
+        if (has_rows) {
+          const uint32_t sc01 = e4m3x2_to_f16x2(sv.x & 0xFFFFu), sc23 = e4m3x2_to_f16x2(sv.x >> 16);
+          const uint32_t sc45 = e4m3x2_to_f16x2(sv.y & 0xFFFFu), sc67 = e4m3x2_to_f16x2(sv.y >> 16);
+          const uint32_t scs[4] = {sc01, sc23, sc45, sc67};
 #pragma unroll
-          for (int G = 0; G < kNG; ++G) {
-            if (G < ngroups) {
-              const uint4 *tl = tile;
-              const uint4 bh0 = tl[act_chunk16(G, sp, 0, g, t)];
-              const uint4 bh1 = tl[act_chunk16(G, sp, 1, g, t)];
-              // MMA j = 0, 1 from half 0; j = 2, 3 from half 1
-              mma_16816_f16(d[G], A0[0], B0[0], A0[1], B0[1], bh0.x, bh0.y);
-              mma_16816_f16(d[G], A0[2], B0[2], A0[3], B0[3], bh0.z, bh0.w);
-              mma_16816_f16(d[G], A1[0], B1[0], A1[1], B1[1], bh1.x, bh1.y);
-              mma_16816_f16(d[G], A1[2], B1[2], A1[3], B1[3], bh1.z, bh1.w);
+          for (int jj = 0; jj < 4; ++jj) {
+            uint32_t rr[16];
+            const uint32_t slo = bcast_lo(scs[jj]), shi = bcast_hi(scs[jj]);
+            e2m1x8_to_f16x2(wv[jj].x, rr[0], rr[1], rr[2], rr[3]);
+            e2m1x8_to_f16x2(wv[jj].y, rr[4], rr[5], rr[6], rr[7]);
+            e2m1x8_to_f16x2(wv[jj].z, rr[8], rr[9], rr[10], rr[11]);
+            e2m1x8_to_f16x2(wv[jj].w, rr[12], rr[13], rr[14], rr[15]);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              rr[i] = hmul2(rr[i], slo);
+              rr[8 + i] = hmul2(rr[8 + i], shi);
             }
+            tmem_st16(tbase + lane_base + kAcol + b * 128u + 64u * (uint32_t)h + 16u * (uint32_t)jj, rr);
           }
         }
+        // ---- activations of this chunk -> fp16 B tile (K-major, 128B swizzle)
+        uint8_t *bt = btile + b * kBTile;
+        unsigned range_bad = 0;
 #pragma unroll
-        for (int G = 0; G < kNG; ++G) {
-          if (G < ngroups) {
-            const float c0 = cs[G * 8 + 2 * t], c1 = cs[G * 8 + 2 * t + 1];
-            acc[G][0] = fmaf(d[G][0], c0, acc[G][0]);
-            acc[G][1] = fmaf(d[G][1], c1, acc[G][1]);
-            acc[G][2] = fmaf(d[G][2], c0, acc[G][2]);
-            acc[G][3] = fmaf(d[G][3], c1, acc[G][3]);
+        for (int i = 0; i < 8; ++i) {
+          const int tau = warp + 8 * i;
+          if (tau >= r.ntok) continue;  // warp-uniform
+          uint4 hv;
+          if (MODE == MOE_W4A16) {
+            float f[8];
+            f[0] = bf16_lo(raw[i].x); f[1] = bf16_hi(raw[i].x);
+            f[2] = bf16_lo(raw[i].y); f[3] = bf16_hi(raw[i].y);
+            f[4] = bf16_lo(raw[i].z); f[5] = bf16_hi(raw[i].z);
+            f[6] = bf16_lo(raw[i].w); f[7] = bf16_hi(raw[i].w);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) range_bad |= (fabsf(f[e]) > 65504.0f) ? 1u : 0u;
+            hv.x = pack_f16x2(f[0], f[1]);
+            hv.y = pack_f16x2(f[2], f[3]);
+            hv.z = pack_f16x2(f[4], f[5]);
+            hv.w = pack_f16x2(f[6], f[7]);
+          } else {
+            uint32_t q0, q1, q2, q3;
+            e2m1x8_to_f16x2(raw[i].x, q0, q1, q2, q3);
+            const uint32_t sc = bcast_lo(e4m3x2_to_f16x2(raw[i].y));
+            hv.x = hmul2(q0, sc);
+            hv.y = hmul2(q1, sc);
+            hv.z = hmul2(q2, sc);
+            hv.w = hmul2(q3, sc);
           }
+          const int katom = lane >> 3, cidx = lane & 7;
+          *reinterpret_cast<uint4 *>(bt + katom * kKatomBytes + tau * 128 + ((cidx ^ (tau & 7)) * 16)) = hv;
+        }
+        if (MODE == MOE_W4A16 && range_bad) raise_device_error(MOE_DEVERR_ACT_RANGE);
+        // prefetch the next chunk's activations (or the next round's first chunk)
+        if (c + 1 < nchunks) {
+          load_act(pair_cur, r.ntok, c + 1);
+        } else if (have_n) {
+          load_act(pair_nxt, rn.ntok, 0);
+        }
+        // ---- publish A (TMEM) and B (shared memory) of item it; release stage s
+        tmem_wait_st();
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&empty[s]);
+          mbar_arrive(&a_full[b]);
+        }
+        // ---- the previous round's epilogue overlaps this round's first chunk
+        if (c == 0 && ep_pending) {
+          epilogue(rp, rnd_p);
+          ep_pending = false;
         }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
+      rp = r;
+      rnd_p = rnd;
+      ep_pending = true;
+      ++rnd;
+      r = rn;
+      pair_cur = pair_nxt;
+      have = have_n;
+      have_n = have && iter.next(meta, RB, rn);
     }
+    if (ep_pending) epilogue(rp, rnd_p);
+  }
 
-    // ---- round epilogue: scale, round to bf16, transpose, 16-byte stores
-    if (has_rows && !*abort_flag) {
-      const float gw = p.w_global ? p.w_global[r.e] : 1.0f;
-      const float f = __fmul_rn(gw, p.g_a);
-      uint16_t *st = staging + cw * (kTS * 16);
-#pragma unroll
-      for (int G = 0; G < kNG; ++G) {
-        if (G < ngroups) {
-          const int c0 = G * 8 + 2 * t;
-          const uint32_t lo = pack_bf16x2(acc[G][0] * f, acc[G][1] * f);  // row g, cols c0, c0+1
-          const uint32_t hi = pack_bf16x2(acc[G][2] * f, acc[G][3] * f);  // row g+8
-          st[c0 * 16 + g] = (uint16_t)(lo & 0xFFFFu);
-          st[(c0 + 1) * 16 + g] = (uint16_t)(lo >> 16);
-          st[c0 * 16 + g + 8] = (uint16_t)(hi & 0xFFFFu);
-          st[(c0 + 1) * 16 + g + 8] = (uint16_t)(hi >> 16);
-        }
-      }
-      __syncwarp();
-      const int nw = r.n0 + cw * 16;
-      for (int task = lane; task < r.ntok * 2; task += 32) {
-        const int col = task >> 1, half = task & 1;
-        const int n = nw + half * 8;
-        if (n < N) {
-          const uint32_t pair = p.order[r.tok0 + col];
-          *reinterpret_cast<uint4 *>(p.out + (int64_t)pair * N + n) =
-              *reinterpret_cast<const uint4 *>(st + col * 16 + half * 8);
-        }
-      }
-      __syncwarp();
-    }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tbase, kTmemCols);
   }
 }
 

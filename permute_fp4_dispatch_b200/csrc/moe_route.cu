@@ -5,8 +5,11 @@
 // choose the kernel variant and launch configuration, enqueue on the
 // caller's stream.  No allocation, no synchronisation (except in
 // moe_get_device_error).
+#include <cudaTypedefs.h>
+
 #include <cstdio>
 #include <cstdlib>
+#include <cstring>
 #include <mutex>
 
 #include "combine.cuh"
@@ -80,6 +83,79 @@ moe_status_t set_smem(Kernel k, size_t bytes) {
 }
 
 int64_t tiles_for(int64_t S) { return (S + moe::idx::kTileSlots - 1) / moe::idx::kTileSlots; }
+
+// ---------------------------------------------------------------- TMA descriptors
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    else
+      cudaGetLastError();
+  });
+  return fn;
+}
+
+// 3-D uint8 map over [E][rows][cols] (cols innermost) with a box of
+// box_cols x box_rows x 1.
+bool encode_u8_3d(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows, uint64_t E,
+                  uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swizzle) {
+  auto fn = tensor_map_encoder();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {cols, rows, E};
+  const cuuint64_t strides[2] = {cols, cols * rows};
+  const cuuint32_t box[3] = {box_cols, box_rows, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Descriptors of the expert library, cached by (pointers, shape): encoding
+// costs a driver call, and graph replays reuse the captured parameters anyway.
+struct LibMaps {
+  const void *w = nullptr, *sfw = nullptr;
+  int E = 0, N = 0, K = 0;
+  bool sf_tma = false;
+  CUtensorMap tw, tsf;
+};
+constexpr int kMapCache = 8;
+LibMaps g_maps[kMapCache];
+int g_maps_next = 0;
+std::mutex g_maps_mu;
+
+bool library_maps(const uint8_t *w, const uint8_t *sfw, int E, int N, int K, LibMaps *out) {
+  std::lock_guard<std::mutex> lock(g_maps_mu);
+  for (auto &m : g_maps)
+    if (m.w == w && m.sfw == sfw && m.E == E && m.N == N && m.K == K) {
+      *out = m;
+      return true;
+    }
+  LibMaps m;
+  m.w = w;
+  m.sfw = sfw;
+  m.E = E;
+  m.N = N;
+  m.K = K;
+  m.sf_tma = (K % 256) == 0;
+  std::memset(&m.tsf, 0, sizeof m.tsf);
+  using namespace moe::gemv;
+  if (!encode_u8_3d(&m.tw, w, (uint64_t)K / 2, (uint64_t)N, (uint64_t)E, kWStride, 16,
+                    CU_TENSOR_MAP_SWIZZLE_128B))
+    return false;
+  if (m.sf_tma && !encode_u8_3d(&m.tsf, sfw, (uint64_t)K / 16, (uint64_t)N, (uint64_t)E,
+                                kSFStride, 16, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return false;
+  g_maps[g_maps_next] = m;
+  g_maps_next = (g_maps_next + 1) % kMapCache;
+  *out = m;
+  return true;
+}
 
 }  // namespace
 
@@ -204,7 +280,8 @@ moe_status_t moe_dispatch_mxfp4(const void *input_tokens, int32_t N, int32_t K, 
   moe_status_t st = check_device(&sms);
   if (st != MOE_OK) return st;
   const int wpb = moe::disp::kWarpsPerBlock;
-  int64_t blocks = ((int64_t)N + wpb - 1) / wpb;
+  const int64_t groups = ((K + 255) / 256 + moe::disp::kSegGroup - 1) / moe::disp::kSegGroup;
+  int64_t blocks = ((int64_t)N * groups + wpb - 1) / wpb;
   if (blocks < 1) blocks = 1;
   if (blocks > (int64_t)sms * 16) blocks = (int64_t)sms * 16;
   moe::disp::dispatch_mxfp4_kernel<<<(unsigned)blocks, wpb * 32, 0, s>>>(
@@ -306,14 +383,15 @@ moe_status_t moe_grouped_gemv_nvfp4(moe_gemv_mode_t mode, const void *act, const
   p.eids = expert_ids;
   p.stats = expert_usage_stats;
   p.out = static_cast<uint16_t *>(out);
-  const bool sf_bulk = (K % 256) == 0;
-  void (*kern)(const Params);
+  LibMaps maps;
+  if (!library_maps(w, sfw, E, N, K, &maps)) return MOE_ERR_CUDA;
+  void (*kern)(const Params, const CUtensorMap, const CUtensorMap);
   if (mode == MOE_W4A16)
-    kern = sf_bulk ? grouped_gemv_kernel<MOE_W4A16, true> : grouped_gemv_kernel<MOE_W4A16, false>;
+    kern = maps.sf_tma ? grouped_gemv_kernel<MOE_W4A16, true> : grouped_gemv_kernel<MOE_W4A16, false>;
   else
-    kern = sf_bulk ? grouped_gemv_kernel<MOE_W4A4, true> : grouped_gemv_kernel<MOE_W4A4, false>;
+    kern = maps.sf_tma ? grouped_gemv_kernel<MOE_W4A4, true> : grouped_gemv_kernel<MOE_W4A4, false>;
   if ((st = set_smem(kern, kSmemBytes)) != MOE_OK) return st;
-  kern<<<(unsigned)sms, kThreads, kSmemBytes, s>>>(p);
+  kern<<<(unsigned)sms, kThreads, kSmemBytes, s>>>(p, maps.tw, maps.tsf);
   return launch_status();
 }
 

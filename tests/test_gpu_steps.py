@@ -291,6 +291,20 @@ def test_gemv_token_major_equals_flattened_pairs():
                                   host_bf16_bits(pipe.expert_out).reshape(-1))
 
 
+def test_gemv_activation_range_is_reported():
+    cfg = wl.small_config("range", N=4, real=4, K=128, E=2, top_k=1, N_out=16)
+    x = wl.activations_bf16(cfg)
+    x[1, 5] = wl.f32_to_bf16_bits(np.array([1.0e5], np.float32))[0]   # beyond fp16 range
+    pipe = RoutingPipeline(cfg.N, cfg.K, cfg.E, cfg.top_k, cfg.N_out, dispatch=False)
+    load_inputs(pipe, cfg, x, wl.routing(cfg), wl.router_weights(cfg))
+    quantize_all_weights(pipe, cfg)
+    assert moe.moe_get_device_error(clear=True) == 0
+    pipe.mask()
+    pipe.create_indices()
+    pipe.gemv()
+    assert moe.moe_get_device_error(clear=True) & moe.MOE_DEVERR_ACT_RANGE
+
+
 def test_gemv_all_slots_unrouted():
     cfg = wl.small_config("empty", N=8, real=0, K=128, E=4, top_k=2, N_out=32)
     pipe, x, ids = run_gemv_case(cfg, "w4a16")
