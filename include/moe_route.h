@@ -120,6 +120,36 @@ MOE_API moe_status_t moe_create_indices(const int64_t *topk_ids, int64_t num_slo
                                 uint32_t *expert_usage_stats, uint32_t *scales_offset,
                                 void *workspace, size_t ws_bytes, cudaStream_t s);
 
+/* The same grouping for callers that cannot provide a workspace.  (The   */
+/* method's pages have no counterpart: this is an interface convenience.) */
+/* Some hosts only hand a kernel its input and output tensors -- plugin  */
+/* interfaces with no allocator or workspace argument, and serving loops */
+/* that freeze their device-memory plan at start-up and forbid any later */
+/* cudaMalloc, which can synchronise the device.  This entry point takes */
+/* no workspace and allocates nothing: its scratch is a fixed array of   */
+/* MOE_CREATE_INDICES_STATIC_SCRATCH bytes inside the library, held by   */
+/* every GPU that loads the library until the process exits.            */
+/*   - Same arguments and outputs as moe_create_indices, minus workspace. */
+/*   - Requires moe_create_indices_workspace_bytes(num_slots, E) <=       */
+/*     MOE_CREATE_INDICES_STATIC_SCRATCH, else MOE_ERR_WORKSPACE and no   */
+/*     launch (E = 64 allows about 8 million slots, E = 1024 half a      */
+/*     million).                                                         */
+/*   - All calls on a device share the one scratch array, and it keeps   */
+/*     the previous call's contents; calls whose kernels may overlap on  */
+/*     the GPU (several streams, several host threads) race on it and    */
+/*     must be serialised by the caller.                                 */
+/*   - The first call on each device looks up the array's device address */
+/*     (cudaGetSymbolAddress, with that device current); make that first */
+/*     call before starting any stream capture.                          */
+#define MOE_CREATE_INDICES_STATIC_SCRATCH ((size_t)262144)
+MOE_API moe_status_t moe_create_indices_static(const int64_t *topk_ids, int64_t num_slots,
+                                               int32_t E, uint32_t *token_expert_order,
+                                               uint32_t *expert_start_indices,
+                                               uint32_t *restore_token_order,
+                                               int32_t *expert_ids,
+                                               uint32_t *expert_usage_stats,
+                                               uint32_t *scales_offset, cudaStream_t s);
+
 /* --------------------------------------------------------------------- */
 /* Step 3 -- MAX "Struct_ep_dispatch_async_mxfp4", execute(), reduced to */
 /* one GPU (n_gpus_per_node = n_nodes = 1: the send buffer is the        */

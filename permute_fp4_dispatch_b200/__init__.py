@@ -22,6 +22,7 @@ __all__ = [
     "MOE_W4A16", "MOE_W4A4", "MOE_EPI_NONE", "MOE_EPI_IDENTITY", "MOE_EPI_SCALE",
     "MOE_DEVERR_WAIT_TIMEOUT", "MOE_DEVERR_RECV_OVERFLOW", "MOE_DEVERR_ACT_RANGE",
     "moe_mask_padding", "moe_create_indices_workspace_bytes", "moe_create_indices",
+    "moe_create_indices_static", "MOE_CREATE_INDICES_STATIC_SCRATCH",
     "moe_mxfp4_row_stride", "moe_dispatch_mxfp4", "moe_quantize_activations_nvfp4",
     "moe_quantize_weights_nvfp4", "moe_grouped_gemv_nvfp4", "moe_combine",
     "moe_status_string", "moe_get_device_error", "moe_version",
@@ -50,6 +51,7 @@ _SIGS = {
     "moe_mask_padding": ([_P, _I32, _I32, _P, _I32, _P], _I32),
     "moe_create_indices_workspace_bytes": ([_I64, _I32], _SZ),
     "moe_create_indices": ([_P, _I64, _I32, _P, _P, _P, _P, _P, _P, _P, _SZ, _P], _I32),
+    "moe_create_indices_static": ([_P, _I64, _I32, _P, _P, _P, _P, _P, _P, _P], _I32),
     "moe_mxfp4_row_stride": ([_I32], _SZ),
     "moe_dispatch_mxfp4": ([_P, _I32, _I32, _I32, _I32, _P, _P, _P, _P, _P, _I64, _P, _P], _I32),
     "moe_quantize_activations_nvfp4": ([_P, _I32, _I32, _F32, _P, _P, _P], _I32),
@@ -130,6 +132,20 @@ def moe_create_indices(topk_ids, num_slots: int, E: int, token_expert_order,
         _ptr(topk_ids), num_slots, E, _ptr(token_expert_order), _ptr(expert_start_indices),
         _ptr(restore_token_order), _ptr(expert_ids), _ptr(expert_usage_stats),
         _ptr(scales_offset), _ptr(workspace), ws_bytes, _stream(stream)), "moe_create_indices")
+
+
+MOE_CREATE_INDICES_STATIC_SCRATCH = 262144
+
+
+def moe_create_indices_static(topk_ids, num_slots: int, E: int, token_expert_order,
+                              expert_start_indices, restore_token_order, expert_ids,
+                              expert_usage_stats, scales_offset, stream=None):
+    """moe_create_indices without a workspace: the scratch is a fixed array inside the
+    library (see include/moe_route.h for the size limit and the sharing rules)."""
+    _check(library().moe_create_indices_static(
+        _ptr(topk_ids), num_slots, E, _ptr(token_expert_order), _ptr(expert_start_indices),
+        _ptr(restore_token_order), _ptr(expert_ids), _ptr(expert_usage_stats),
+        _ptr(scales_offset), _stream(stream)), "moe_create_indices_static")
 
 
 def moe_mxfp4_row_stride(K: int) -> int:

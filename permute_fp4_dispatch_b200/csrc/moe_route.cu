@@ -427,3 +427,54 @@ moe_status_t moe_combine(const void *expert_out, const float *router_weights,
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------ no-allocation grouping
+// Scratch of moe_create_indices_static: a fixed array in the library's own
+// device memory, so callers that cannot allocate still get the tiled path.
+// Host code must not pass the symbol itself to a kernel (on the host it only
+// names a host-side shadow); the device address is looked up once per device.
+namespace {
+static __device__ __align__(256) unsigned char g_create_indices_scratch[MOE_CREATE_INDICES_STATIC_SCRATCH];
+void *g_scratch_addr[kMaxDevices];
+std::mutex g_scratch_mu;
+
+moe_status_t static_scratch(void **out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_addr[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_create_indices_scratch) != cudaSuccess || !p) {
+      cudaGetLastError();
+      return MOE_ERR_CUDA;
+    }
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return MOE_OK;
+}
+}  // namespace
+
+extern "C" moe_status_t moe_create_indices_static(const int64_t *topk_ids, int64_t num_slots,
+                                                  int32_t E, uint32_t *token_expert_order,
+                                                  uint32_t *expert_start_indices,
+                                                  uint32_t *restore_token_order,
+                                                  int32_t *expert_ids,
+                                                  uint32_t *expert_usage_stats,
+                                                  uint32_t *scales_offset, cudaStream_t s) {
+  if (E < 1 || E > 1024 || num_slots < 0 || num_slots >= (int64_t(1) << 31))
+    return MOE_ERR_INVALID_ARG;
+  if (moe_create_indices_workspace_bytes(num_slots, E) > MOE_CREATE_INDICES_STATIC_SCRATCH)
+    return MOE_ERR_WORKSPACE;
+  moe_status_t st = check_device();
+  if (st != MOE_OK) return st;
+  void *scratch = nullptr;
+  if ((st = static_scratch(&scratch)) != MOE_OK) return st;
+  return moe_create_indices(topk_ids, num_slots, E, token_expert_order, expert_start_indices,
+                            restore_token_order, expert_ids, expert_usage_stats, scales_offset,
+                            scratch, MOE_CREATE_INDICES_STATIC_SCRATCH, s);
+}

@@ -52,6 +52,7 @@ def test_host_validation_runs_before_any_device_work(lib):
     assert lib.moe_mask_padding(P, -1, 2, P, 0, None) == 1
     assert lib.moe_create_indices(P, 8, 0, P, P, P, P, P, None, P, 256, None) == 1
     assert lib.moe_create_indices(P, 8, 4, P, P, P, P, P, None, None, 0, None) == 3
+    assert lib.moe_create_indices_static(P, 8, 2000, P, P, P, P, P, None, None) == 1
     assert lib.moe_dispatch_mxfp4(P, 4, 48, 2, 4, P, P, P, P, P, 8, P, None) == 1   # K % 32
     assert lib.moe_quantize_activations_nvfp4(P, 4, 24, 1.0, P, P, None) == 1      # K % 16
     assert lib.moe_quantize_activations_nvfp4(P, 4, 32, 0.0, P, P, None) == 1      # g > 0
