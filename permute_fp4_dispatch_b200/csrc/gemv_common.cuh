@@ -1,0 +1,102 @@
+// gemv_common.cuh -- shared pieces of the grouped NVFP4 GEMV kernels: launch
+// parameters, the per-CTA work partition over (active expert, token pass,
+// 16-row block) units, and small helpers.
+#pragma once
+#include "common.cuh"
+
+namespace moe {
+namespace gemv {
+
+constexpr int kMaxExperts = 1024;
+constexpr int kBlocksPerRound = 8;      // 16-row blocks per round (128 rows)
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+
+struct Params {
+  const void *act;          // W4A16: bf16 [M, K]; W4A4: u8 [M, K/2]
+  const uint8_t *sfa;       // W4A4: [M, K/16]
+  float g_a;
+  int32_t top_k;
+  const uint8_t *w;         // [E, N, K/2]
+  const uint8_t *sfw;       // [E, N, K/16]
+  const float *w_global;    // [E] or null
+  int32_t N, K;
+  const uint32_t *order;
+  const uint32_t *start;
+  const int32_t *eids;
+  const uint32_t *stats;
+  uint16_t *out;            // bf16 [M, top_k, N]
+};
+
+struct Round {
+  int e;
+  uint32_t tok0;
+  int ntok;
+  int n0;
+  int nrows;
+  int nblk;
+};
+
+// Per-expert metadata staged in shared memory at kernel start.
+struct Meta {
+  const uint32_t *prefix;  // units before active expert a
+  const uint32_t *start;   // CSR offsets
+  const int32_t *eid;      // expert ids
+  int N;
+};
+
+// Walks a CTA's unit range round by round; identical in every thread.
+struct RoundIter {
+  uint32_t u, u_end;
+  int a;
+  uint32_t ts;  // tokens per pass
+  __device__ __forceinline__ bool next(const Meta &m, int RB, Round &r) {
+    if (u >= u_end) return false;
+    while (u >= m.prefix[a + 1]) ++a;
+    const uint32_t v = u - m.prefix[a];
+    const uint32_t pass = v / (uint32_t)RB;
+    const uint32_t rb = v % (uint32_t)RB;
+    uint32_t nblk = (uint32_t)RB - rb;
+    if (nblk > (uint32_t)kBlocksPerRound) nblk = kBlocksPerRound;
+    if (nblk > u_end - u) nblk = u_end - u;
+    const uint32_t s0 = m.start[a];
+    const uint32_t c = m.start[a + 1] - s0;
+    r.e = m.eid[a];
+    r.tok0 = s0 + pass * ts;
+    r.ntok = (int)min(ts, c - pass * ts);
+    r.n0 = (int)rb * 16;
+    r.nrows = min((int)nblk * 16, m.N - r.n0);
+    r.nblk = (int)nblk;
+    u += nblk;
+    return true;
+  }
+};
+
+__device__ __forceinline__ uint32_t bcast_lo(uint32_t h) { return __byte_perm(h, h, 0x1010); }
+__device__ __forceinline__ uint32_t bcast_hi(uint32_t h) { return __byte_perm(h, h, 0x3232); }
+
+// Warp 0 of the CTA: prefix[a] = units before active expert a, where an
+// expert with c tokens has ceil(c / ts) passes of RB row blocks.
+__device__ __forceinline__ void build_prefix(uint32_t *prefix, const uint32_t *start, uint32_t A,
+                                             uint32_t ts, int RB, int lane) {
+  uint32_t run = 0;
+  for (uint32_t a0 = 0; a0 < A; a0 += 32) {
+    const uint32_t a = a0 + lane;
+    uint32_t units = 0;
+    if (a < A) {
+      const uint32_t c = start[a + 1] - start[a];
+      units = (c + ts - 1) / ts * (uint32_t)RB;
+    }
+    uint32_t x = units;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (a < A) prefix[a + 1] = run + x;
+    run += __shfl_sync(0xffffffffu, x, 31);
+  }
+  if (lane == 0) prefix[0] = 0;
+}
+
+}  // namespace gemv
+}  // namespace moe

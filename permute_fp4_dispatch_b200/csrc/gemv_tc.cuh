@@ -1,4 +1,5 @@
-// gemv_nvfp4.cuh -- step 4b: grouped expert GEMV on an NVFP4 expert library.
+// gemv_tc.cuh -- step 4b, tensor-memory variant: grouped expert GEMV on an
+// NVFP4 expert library, for passes of many tokens per expert.
 //
 // FlashRT "grouped-moe-gemv" card (Available functions:
 // grouped_w4a16_gemv_bf16 / grouped_w4a4_gemv_bf16; W4A4 routing is
@@ -40,16 +41,16 @@
 //     <= 2^-25) below; |x| > 65504 raises MOE_DEVERR_ACT_RANGE.  W4A4
 //     activations are dequantised exactly like the weights.
 #pragma once
-#include "common.cuh"
+#include "gemv_common.cuh"
 
 namespace moe {
 namespace gemv {
+namespace tc {
 
 constexpr int kDQ = 8;                  // dequant / staging / epilogue warps
 constexpr int kTmaWarp = kDQ;
 constexpr int kMmaWarp = kDQ + 1;
 constexpr int kThreads = (kDQ + 2) * 32;
-constexpr int kBlocksPerRound = 8;      // 16-row blocks per round (M = 128)
 constexpr int kKC = 256;                // columns (codes) per chunk
 constexpr int kTS = 64;                 // tokens per pass (MMA N <= 64)
 constexpr int kStages = 5;
@@ -61,11 +62,9 @@ constexpr int kStageW = 128 * kWStride;
 constexpr int kStageBytes = kStageW + 128 * kSFStride;
 constexpr int kKatomBytes = kTS * 128;  // one 64-column slab of the B tile
 constexpr int kBTile = 4 * kKatomBytes;
-constexpr int kMaxExperts = 1024;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAcol = 0;           // A tiles: columns [0, 256), 128 per buffer
 constexpr uint32_t kDcol = 256;         // D tiles: columns [256, 384), 64 per buffer
-constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
 static_assert(kStageBytes % 1024 == 0, "stages must keep the 1024-byte swizzle alignment");
 constexpr size_t kOffB = (size_t)kStages * kStageBytes;
@@ -77,68 +76,6 @@ constexpr size_t kOffBar = kOffPair + 2 * kTS * 4;
 constexpr int kNumBars = 2 * kStages + 8;
 constexpr size_t kOffMisc = kOffBar + kNumBars * 8;             // tmem slot, abort flag
 constexpr size_t kSmemBytes = kOffMisc + 16 + 1024;             // + alignment slack
-
-struct Params {
-  const void *act;          // W4A16: bf16 [M, K]; W4A4: u8 [M, K/2]
-  const uint8_t *sfa;       // W4A4: [M, K/16]
-  float g_a;
-  int32_t top_k;
-  const uint8_t *w;         // [E, N, K/2]
-  const uint8_t *sfw;       // [E, N, K/16]
-  const float *w_global;    // [E] or null
-  int32_t N, K;
-  const uint32_t *order;
-  const uint32_t *start;
-  const int32_t *eids;
-  const uint32_t *stats;
-  uint16_t *out;            // bf16 [M, top_k, N]
-};
-
-struct Round {
-  int e;
-  uint32_t tok0;
-  int ntok;
-  int n0;
-  int nrows;
-  int nblk;
-};
-
-// Per-expert metadata staged in shared memory at kernel start.
-struct Meta {
-  const uint32_t *prefix;  // units before active expert a
-  const uint32_t *start;   // CSR offsets
-  const int32_t *eid;      // expert ids
-  int N;
-};
-
-// Walks a CTA's unit range round by round; identical in every thread.
-struct RoundIter {
-  uint32_t u, u_end;
-  int a;
-  __device__ __forceinline__ bool next(const Meta &m, int RB, Round &r) {
-    if (u >= u_end) return false;
-    while (u >= m.prefix[a + 1]) ++a;
-    const uint32_t v = u - m.prefix[a];
-    const uint32_t pass = v / (uint32_t)RB;
-    const uint32_t rb = v % (uint32_t)RB;
-    uint32_t nblk = (uint32_t)RB - rb;
-    if (nblk > (uint32_t)kBlocksPerRound) nblk = kBlocksPerRound;
-    if (nblk > u_end - u) nblk = u_end - u;
-    const uint32_t s0 = m.start[a];
-    const uint32_t c = m.start[a + 1] - s0;
-    r.e = m.eid[a];
-    r.tok0 = s0 + pass * kTS;
-    r.ntok = (int)min((uint32_t)kTS, c - pass * kTS);
-    r.n0 = (int)rb * 16;
-    r.nrows = min((int)nblk * 16, m.N - r.n0);
-    r.nblk = (int)nblk;
-    u += nblk;
-    return true;
-  }
-};
-
-__device__ __forceinline__ uint32_t bcast_lo(uint32_t h) { return __byte_perm(h, h, 0x1010); }
-__device__ __forceinline__ uint32_t bcast_hi(uint32_t h) { return __byte_perm(h, h, 0x3232); }
 
 template <int MODE, bool SF_TMA>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -167,31 +104,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int RB = (N + 15) / 16;
   const uint32_t A = p.stats[1];
 
-  // units per active expert = passes * row blocks; prefix over experts
-  if (warp == 0) {
-    uint32_t run = 0;
-    for (uint32_t a0 = 0; a0 < A; a0 += 32) {
-      const uint32_t a = a0 + lane;
-      uint32_t units = 0;
-      if (a < A) {
-        const uint32_t c = p.start[a + 1] - p.start[a];
-        units = (c + kTS - 1) / kTS * (uint32_t)RB;
-      }
-      uint32_t x = units;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
-      }
-      if (a < A) prefix[a + 1] = run + x;
-      run += __shfl_sync(0xffffffffu, x, 31);
-    }
-    if (lane == 0) prefix[0] = 0;
-  }
   for (uint32_t i = threadIdx.x; i <= A; i += blockDim.x) {
     s_start[i] = p.start[i];
     if (i < A) s_eid[i] = p.eids[i];
   }
+  __syncthreads();
+  if (warp == 0) build_prefix(prefix, s_start, A, kTS, RB, lane);
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], SF_TMA ? 1u : 33u);
@@ -226,7 +144,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == kTmaWarp) {
     // ================================================================ TMA producer
-    RoundIter iter{u_begin, u_end, 0};
+    RoundIter iter{u_begin, u_end, 0, (uint32_t)kTS};
     Round r;
     uint32_t it = 0;
     const uint64_t policy = l2_evict_first_policy();
@@ -264,7 +182,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kMmaWarp) {
     // ================================================================ MMA issuer
     if (lane == 0) {
-      RoundIter iter{u_begin, u_end, 0};
+      RoundIter iter{u_begin, u_end, 0, (uint32_t)kTS};
       Round r;
       uint32_t it = 0, rnd = 0;
       while (iter.next(meta, RB, r)) {
@@ -302,7 +220,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int h = warp >> 2;    // column half of a chunk
     const int row = 32 * q + lane;
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-    RoundIter iter{u_begin, u_end, 0};
+    RoundIter iter{u_begin, u_end, 0, (uint32_t)kTS};
     Round r, rn, rp;  // current, next, previous (pending epilogue)
     bool have = iter.next(meta, RB, r);
     bool have_n = have && iter.next(meta, RB, rn);
@@ -507,5 +425,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+}  // namespace tc
 }  // namespace gemv
 }  // namespace moe

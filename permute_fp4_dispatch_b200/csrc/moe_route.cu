@@ -16,7 +16,8 @@
 #include "common.cuh"
 #include "create_indices.cuh"
 #include "dispatch_mxfp4.cuh"
-#include "gemv_nvfp4.cuh"
+#include "gemv_mma.cuh"
+#include "gemv_tc.cuh"
 #include "mask.cuh"
 #include "quant_nvfp4.cuh"
 
@@ -144,12 +145,14 @@ bool library_maps(const uint8_t *w, const uint8_t *sfw, int E, int N, int K, Lib
   m.K = K;
   m.sf_tma = (K % 256) == 0;
   std::memset(&m.tsf, 0, sizeof m.tsf);
-  using namespace moe::gemv;
-  if (!encode_u8_3d(&m.tw, w, (uint64_t)K / 2, (uint64_t)N, (uint64_t)E, kWStride, 16,
+  // both GEMV variants read 16-row x 128-byte weight boxes and 16-row x 16-byte scale boxes
+  static_assert(moe::gemv::tc::kWStride == 128 && moe::gemv::mma::kWStride == 128, "box width");
+  static_assert(moe::gemv::tc::kSFStride == 16 && moe::gemv::mma::kSFStride == 16, "box width");
+  if (!encode_u8_3d(&m.tw, w, (uint64_t)K / 2, (uint64_t)N, (uint64_t)E, 128, 16,
                     CU_TENSOR_MAP_SWIZZLE_128B))
     return false;
-  if (m.sf_tma && !encode_u8_3d(&m.tsf, sfw, (uint64_t)K / 16, (uint64_t)N, (uint64_t)E,
-                                kSFStride, 16, CU_TENSOR_MAP_SWIZZLE_NONE))
+  if (m.sf_tma && !encode_u8_3d(&m.tsf, sfw, (uint64_t)K / 16, (uint64_t)N, (uint64_t)E, 16, 16,
+                                CU_TENSOR_MAP_SWIZZLE_NONE))
     return false;
   g_maps[g_maps_next] = m;
   g_maps_next = (g_maps_next + 1) % kMapCache;
@@ -363,7 +366,7 @@ moe_status_t moe_grouped_gemv_nvfp4(moe_gemv_mode_t mode, const void *act, const
     return MOE_ERR_INVALID_ARG;
   // the flat unit count must fit 32 bits: (S / 32 + E) * ceil(N / 16)
   const int64_t S = (int64_t)M * top_k;
-  if ((S / kTS + E + 1) * ((N + 15) / 16) >= (int64_t(1) << 32)) return MOE_ERR_INVALID_ARG;
+  if ((S / 8 + E + 1) * ((N + 15) / 16) >= (int64_t(1) << 32)) return MOE_ERR_INVALID_ARG;
   int sms = 0;
   moe_status_t st = check_device(&sms);
   if (st != MOE_OK) return st;
@@ -385,13 +388,37 @@ moe_status_t moe_grouped_gemv_nvfp4(moe_gemv_mode_t mode, const void *act, const
   p.out = static_cast<uint16_t *>(out);
   LibMaps maps;
   if (!library_maps(w, sfw, E, N, K, &maps)) return MOE_ERR_CUDA;
+  // Decode-sized passes (few tokens per expert on average) take the register-
+  // dequant mma.sync variant; many tokens per expert take the tensor-memory
+  // variant, whose tcgen05 MMA has a fixed per-instruction cost up to N = 64.
+  const int ts_mma = mma::tokens_per_pass(K);
+  bool use_mma = ts_mma >= 8 && (S / E) < 48;
+  // test hook: MOE_GEMV_VARIANT=mma|tc forces a variant (both are exact for every input)
+  if (const char *v = std::getenv("MOE_GEMV_VARIANT")) {
+    if (v[0] == 'm' && ts_mma >= 8) use_mma = true;
+    if (v[0] == 't') use_mma = false;
+  }
+  if (use_mma) {
+    void (*kern)(const Params, const int, const CUtensorMap, const CUtensorMap);
+    if (mode == MOE_W4A16)
+      kern = maps.sf_tma ? mma::grouped_gemv_mma_kernel<MOE_W4A16, true>
+                         : mma::grouped_gemv_mma_kernel<MOE_W4A16, false>;
+    else
+      kern = maps.sf_tma ? mma::grouped_gemv_mma_kernel<MOE_W4A4, true>
+                         : mma::grouped_gemv_mma_kernel<MOE_W4A4, false>;
+    if ((st = set_smem(kern, mma::kSmemBytes)) != MOE_OK) return st;
+    kern<<<(unsigned)sms, mma::kThreads, mma::kSmemBytes, s>>>(p, ts_mma, maps.tw, maps.tsf);
+    return launch_status();
+  }
   void (*kern)(const Params, const CUtensorMap, const CUtensorMap);
   if (mode == MOE_W4A16)
-    kern = maps.sf_tma ? grouped_gemv_kernel<MOE_W4A16, true> : grouped_gemv_kernel<MOE_W4A16, false>;
+    kern = maps.sf_tma ? tc::grouped_gemv_kernel<MOE_W4A16, true>
+                       : tc::grouped_gemv_kernel<MOE_W4A16, false>;
   else
-    kern = maps.sf_tma ? grouped_gemv_kernel<MOE_W4A4, true> : grouped_gemv_kernel<MOE_W4A4, false>;
-  if ((st = set_smem(kern, kSmemBytes)) != MOE_OK) return st;
-  kern<<<(unsigned)sms, kThreads, kSmemBytes, s>>>(p, maps.tw, maps.tsf);
+    kern = maps.sf_tma ? tc::grouped_gemv_kernel<MOE_W4A4, true>
+                       : tc::grouped_gemv_kernel<MOE_W4A4, false>;
+  if ((st = set_smem(kern, tc::kSmemBytes)) != MOE_OK) return st;
+  kern<<<(unsigned)sms, tc::kThreads, tc::kSmemBytes, s>>>(p, maps.tw, maps.tsf);
   return launch_status();
 }
 

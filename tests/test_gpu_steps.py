@@ -249,8 +249,16 @@ def run_gemv_case(cfg, mode, act_global=1.0):
     return pipe, x, oracle.mask_padding(ids, cfg.real)
 
 
+@pytest.fixture(params=["auto", "mma", "tc"])
+def gemv_variant(request, monkeypatch):
+    """Run a GEMV case through the host's choice and through each kernel variant."""
+    if request.param != "auto":
+        monkeypatch.setenv("MOE_GEMV_VARIANT", request.param)
+    yield request.param
+
+
 @pytest.mark.parametrize("name,cfg,mode", GEMV_CASES, ids=[c[0] for c in GEMV_CASES])
-def test_gemv_parity(name, cfg, mode):
+def test_gemv_parity(name, cfg, mode, gemv_variant):
     g_a = 1.0 if mode == "w4a16" else float(np.float32(0.5))
     pipe, x, ids = run_gemv_case(cfg, mode, g_a)
     wq, sfw, gw = oracle_weights(cfg, range(cfg.E))
@@ -271,7 +279,7 @@ def test_gemv_parity(name, cfg, mode):
     assert_float_parity(host_bf16_f64(pipe.expert_out)[routed], ref[routed], what=name)
 
 
-def test_gemv_token_major_equals_flattened_pairs():
+def test_gemv_token_major_equals_flattened_pairs(gemv_variant):
     cfg = wl.small_config("flat", N=50, real=44, K=320, E=7, top_k=4, N_out=136)
     pipe, x, ids = run_gemv_case(cfg, "w4a16")
     # same pairs as a [R, 1] map: one activation row per (token, slot)
