@@ -6,10 +6,11 @@
 // restore_token_order[p] (from moe_create_indices), so no slot claiming is
 // needed and the row order is deterministic.
 //
-// One warp per (token, group of up to 8 segments of 256 columns): the row is
-// read once (128-bit loads, 8 bf16 per lane, all of the group's loads in
-// flight together), encoded once, and the encoded 32-bit words are stored to
-// each of the token's routed rows.  A 32-element MX block is 4 lanes; its
+// One warp per (token, group of SEG segments of 256 columns): the row is read
+// once (128-bit loads, 8 bf16 per lane, all of the group's loads in flight
+// together), encoded once, and the encoded 32-bit words are stored to each of
+// the token's routed rows.  The host picks SEG (8, 4, 2 or 1) so that even a
+// decode batch of a hundred tokens spreads over every SM.  A 32-element MX block is 4 lanes; its
 // amax is a 2-step xor-shuffle.  Padding tokens (no routed slot) write
 // nothing.
 #pragma once
@@ -19,7 +20,6 @@ namespace moe {
 namespace disp {
 
 constexpr int kWarpsPerBlock = 8;
-constexpr int kSegGroup = 8;  // 256-column segments per warp task
 
 // E8M0 exponent of a block: floor(log2(amax)) - 2 clamped to [-127, 127];
 // amax == 0 gives -127.  Exact integer arithmetic on the fp32 bits.
@@ -39,6 +39,7 @@ __device__ __forceinline__ int mx_shared_exponent(float amax) {
   return se;
 }
 
+template <int SEG>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     dispatch_mxfp4_kernel(const uint16_t *__restrict__ x, int32_t N, int32_t K, int32_t top_k,
                           int32_t E, const uint32_t *__restrict__ restore,
@@ -58,7 +59,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
   const int half = K / 2;
   const int nscale = K / 32;
   const int segs = (K + 255) / 256;
-  const int groups = (segs + kSegGroup - 1) / kSegGroup;
+  const int groups = (segs + SEG - 1) / SEG;
   const int64_t tasks = (int64_t)N * groups;
   for (int64_t task = (int64_t)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5); task < tasks;
        task += warps_total) {
@@ -66,10 +67,10 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     const int grp = (int)(task % groups);
     const uint16_t *row = x + (int64_t)t * K;
     // issue the group's row loads first (independent of the destinations)
-    uint4 v[kSegGroup];
+    uint4 v[SEG];
 #pragma unroll
-    for (int q = 0; q < kSegGroup; ++q) {
-      const int k = (grp * kSegGroup + q) * 256 + 8 * (int)lane;
+    for (int q = 0; q < SEG; ++q) {
+      const int k = (grp * SEG + q) * 256 + 8 * (int)lane;
       v[q] = k < K ? ldg_nc_v4(row + k) : make_uint4(0u, 0u, 0u, 0u);
     }
     for (int j0 = 0; j0 < top_k; j0 += 32) {
@@ -85,9 +86,9 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
       const unsigned dmask = __ballot_sync(0xffffffffu, ok);
       if (dmask == 0u) continue;
 #pragma unroll
-      for (int q = 0; q < kSegGroup; ++q) {
-        const int k = (grp * kSegGroup + q) * 256 + 8 * (int)lane;
-        if ((grp * kSegGroup + q) * 256 >= K) break;  // warp-uniform
+      for (int q = 0; q < SEG; ++q) {
+        const int k = (grp * SEG + q) * 256 + 8 * (int)lane;
+        if ((grp * SEG + q) * 256 >= K) break;  // warp-uniform
         const bool active = k < K;
         float f[8];
         f[0] = bf16_lo(v[q].x); f[1] = bf16_hi(v[q].x);

@@ -8,7 +8,8 @@ namespace moe {
 namespace gemv {
 
 constexpr int kMaxExperts = 1024;
-constexpr int kBlocksPerRound = 8;      // 16-row blocks per round (128 rows)
+constexpr int kBlocksPerRound = 8;      // 16-row blocks per round (128 rows), unless a
+                                        // kernel asks for another round size
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
 struct Params {
@@ -49,6 +50,7 @@ struct RoundIter {
   uint32_t u, u_end;
   int a;
   uint32_t ts;  // tokens per pass
+  uint32_t round_blocks = kBlocksPerRound;
   __device__ __forceinline__ bool next(const Meta &m, int RB, Round &r) {
     if (u >= u_end) return false;
     while (u >= m.prefix[a + 1]) ++a;
@@ -56,7 +58,7 @@ struct RoundIter {
     const uint32_t pass = v / (uint32_t)RB;
     const uint32_t rb = v % (uint32_t)RB;
     uint32_t nblk = (uint32_t)RB - rb;
-    if (nblk > (uint32_t)kBlocksPerRound) nblk = kBlocksPerRound;
+    if (nblk > round_blocks) nblk = round_blocks;
     if (nblk > u_end - u) nblk = u_end - u;
     const uint32_t s0 = m.start[a];
     const uint32_t c = m.start[a + 1] - s0;

@@ -1,33 +1,42 @@
 // gemv_mma.cuh -- step 4b, decode variant: grouped expert GEMV on an NVFP4
-// expert library for passes of up to 32 tokens per expert.
+// expert library for passes of up to 16 tokens per expert.
 //
 // FlashRT "grouped-moe-gemv" card (Available functions:
 // grouped_w4a16_gemv_bf16 / grouped_w4a4_gemv_bf16; token-major routing).
 //
 // At decode batch sizes the weight stream is the roofline and the
-// tensor-core work per weight is tiny (8-32 tokens), so this variant keeps
-// the tensor cores fed from registers:
-//   * Same work partition as the tensor-memory variant: (active expert, pass,
-//     16-row block) units in equal contiguous ranges per persistent CTA,
-//     rounds of up to 8 blocks of one (expert, pass).
-//   * Warp 8 streams the FP4 rows and E4M3 scales of each round, 256 columns
-//     per chunk, into a kStages-deep ring with tiled TMA (16-row x 128-byte
-//     boxes, 128-byte swizzle, L2 evict-first).  Warps 0-7 each own 16 rows
-//     of a round and release a stage with an mbarrier arrive when done: the
-//     warps never wait for one another inside a round.
+// tensor-core work per weight is tiny (8-16 tokens), so this variant keeps
+// the tensor cores fed from registers and spends its effort on the stream:
+//   * Work partition shared with the tensor-memory variant: (active expert,
+//     pass, 16-row block) units in equal contiguous ranges per persistent
+//     CTA, rounds of up to 16 blocks of one (expert, pass); warp w owns block
+//     w of every round.
+//   * Every warp runs its own one-stage pipeline, with no producer warp and
+//     no cross-warp waits inside a pass; sixteen warps (four per scheduler)
+//     hide each other's load and dependency latencies.  A stage is 16 rows x
+//     1024 codes:
+//     one 4-D TMA box (16 rows x 4 lines of 128 bytes, 512 contiguous bytes
+//     per row, 128-byte swizzle, L2 evict-first) issued by lane 0, plus the
+//     stage's 16 x 64 E4M3 scale bytes by per-lane 16-byte cp.async, both
+//     completing on the stage's mbarrier.  The TMA engine's cost grows with
+//     the number of contiguous runs it fetches; 512-byte runs stream at the
+//     rate of plain bulk copies where 128-byte runs do not.
+//   * Lane (g, t) owns line t of rows g and g + 8.  A line index in the box is
+//     4 * row + line, so the swizzle key is (row & 1) * 4 + line and the eight
+//     lanes of one shared-memory phase (rows g, g + 1) hit eight distinct
+//     16-byte bank groups.
 //   * When a CTA starts a new (expert, pass), the 8 warps convert that pass's
-//     activation rows once, for the whole K, into an fp16 tile in shared
-//     memory laid out in mma fragment order with an XOR swizzle; every round
-//     of the pass reuses it.  W4A16: plain bf16 -> fp16 (exact for
-//     2^-14 <= |x| <= 65504, MOE_DEVERR_ACT_RANGE beyond); W4A4: E2M1 x E4M3
-//     products, exact in fp16.
-//   * Each lane dequantises its two rows' codes in registers (hardware
-//     E2M1 -> f16x2 converter, times the block's E4M3 scale: exact in fp16)
-//     and issues m16n8k16 MMAs (fp32 accumulation, two independent chains per
-//     8-token group) with the tokens on the n side.  Within a 64-column span
-//     each lane owns 16 contiguous columns (one scale block); A and B use the
-//     same column permutation, so the dot product is unchanged.
-//   * The round's accumulators are scaled by g_w * g_a, rounded to bf16,
+//     activation rows once, for the whole K, into an fp16 tile laid out in
+//     mma fragment order; every round of the pass reuses it.  W4A16: plain
+//     bf16 -> fp16 (exact for 2^-14 <= |x| <= 65504, MOE_DEVERR_ACT_RANGE
+//     beyond); W4A4: E2M1 x E4M3 products, exact in fp16.
+//   * Each lane dequantises its codes in registers (hardware E2M1 -> f16x2
+//     converter, times the block's E4M3 scale: exact in fp16) and issues
+//     m16n8k16 MMAs (fp32 accumulation, two independent chains per 8-token
+//     group) with the tokens on the n side.  Lane t's MMA i takes the four
+//     codes 256 t + 4 i .. + 3 of the stage; the activation tile uses the same
+//     column permutation, so the dot product is unchanged.
+//   * Each block's accumulators are scaled by g_w * g_a, rounded to bf16,
 //     transposed through shared memory and written as 16-byte row segments.
 #pragma once
 #include "gemv_common.cuh"
@@ -36,119 +45,113 @@ namespace moe {
 namespace gemv {
 namespace mma {
 
-constexpr int kCW = 8;                  // compute warps (16 rows each)
-constexpr int kThreads = (kCW + 1) * 32;
-constexpr int kKC = 256;                // columns per chunk
-constexpr int kMaxTS = 32;              // tokens per pass at most (4 groups of 8)
+constexpr int kCW = 16;                      // warps, one 16-row block each per round
+constexpr int kThreads = kCW * 32;
+constexpr int kLines = 4;                    // 128-byte lines (256 codes) per row per stage
+constexpr int kKS = kLines * 256;            // codes per row per stage
+constexpr int kSlots = 1;                    // pipeline stages per warp
+constexpr int kRowW = kLines * 128;          // bytes of codes per row per stage
+constexpr int kRowSF = kLines * 16;          // scale bytes per row per stage
+constexpr int kStageW = 16 * kRowW;          // 8 KB
+constexpr int kStageSF = 16 * kRowSF;        // 1 KB
+constexpr int kMaxTS = 16;                   // tokens per pass at most (2 groups of 8)
 constexpr int kNG = kMaxTS / 8;
-constexpr int kStages = 4;
-constexpr int kWStride = kKC / 2;
-constexpr int kSFStride = kKC / 16;
-constexpr int kBoxW = 16 * kWStride;
-constexpr int kBoxSF = 16 * kSFStride;
-constexpr int kStageW = 128 * kWStride;
-constexpr int kStageBytes = kStageW + 128 * kSFStride;
-constexpr int kGroupChunkBytes = 4 * 2 * 32 * 16;  // one 8-token group x one chunk (4 KB)
-constexpr int kActBytes = 128 * 1024;              // fp16 activation tile of a pass
+constexpr int kGroupStageBytes = 8 * kKS * 2;  // fp16 tile of one 8-token group x one stage
+constexpr int kActBytes = 64 * 1024;
 constexpr int kStagingBytes = kCW * kMaxTS * 16 * 2;
+constexpr uint64_t kDrainLimitNs = 100000000ull;  // 100 ms
 
-static_assert(kStageBytes % 1024 == 0, "stages must keep the 1024-byte swizzle alignment");
-constexpr size_t kOffAct = (size_t)kStages * kStageBytes;
+constexpr size_t kOffW = 0;
+constexpr size_t kOffSF = kOffW + (size_t)kCW * kSlots * kStageW;
+constexpr size_t kOffAct = kOffSF + (size_t)kCW * kSlots * kStageSF;
 constexpr size_t kOffStaging = kOffAct + kActBytes;
 constexpr size_t kOffPrefix = kOffStaging + kStagingBytes;
-constexpr size_t kOffStart = kOffPrefix + (kMaxExperts + 4) * 4;
-constexpr size_t kOffEid = kOffStart + (kMaxExperts + 4) * 4;
-constexpr size_t kOffPair = kOffEid + (kMaxExperts + 4) * 4;
+constexpr size_t kOffPair = kOffPrefix + (kMaxExperts + 4) * 4;
 constexpr size_t kOffBar = kOffPair + kMaxTS * 4;
-constexpr size_t kOffMisc = kOffBar + 2 * kStages * 8;
+constexpr size_t kOffMisc = kOffBar + (size_t)kCW * kSlots * 8;
 constexpr size_t kSmemBytes = kOffMisc + 16 + 1024;
+static_assert(kStageW % 1024 == 0, "stages must keep the 1024-byte swizzle alignment");
+static_assert(kOffBar % 8 == 0, "mbarrier alignment");
+static_assert(kSmemBytes <= 232448, "shared memory per block");
 
-// Tokens per pass for a hidden size K: as many 8-token groups (up to 4) as
-// the activation tile holds for the whole K; 0 when not even one fits.
+// Tokens per pass for a hidden size K (a multiple of 256): as many 8-token
+// groups (up to 2) as the activation tile holds for the whole K; 0 when not
+// even one fits.
 __host__ __device__ constexpr int tokens_per_pass(int K) {
-  const int nchunks = (K + kKC - 1) / kKC;
-  const int groups = kActBytes / (nchunks * kGroupChunkBytes);
+  const int nst = (K + kKS - 1) / kKS;
+  const int groups = kActBytes / (nst * kGroupStageBytes);
   return 8 * (groups < kNG ? groups : kNG);
 }
 
-// fp16 activation tile index (16-byte units): chunk c, group G (of ng), span s,
-// half h, lane (g, t).
-__device__ __forceinline__ int act_index(int c, int ng, int G, int s, int h, int g, int t) {
-  return ((((c * ng + G) * 4 + s) * 2 + h) * 32) + ((g * 4 + t) ^ (2 * s + h));
+// fp16 activation tile index (16-byte units): stage c, group G (of ng), MMA
+// pair m (MMAs 2m, 2m + 1 of the stage), lane (g, t) = 4 g + t.
+__device__ __forceinline__ int act_index(int c, int ng, int G, int m, int lane) {
+  return (((c * ng + G) * 32 + m) << 5) + lane;
 }
 
-// One chunk of one warp: dequantise its two rows' 256 codes (lane (g, t):
-// rows g and g + 8, columns 64t..64t+63 of the chunk), multiply with the NG
-// token groups of the activation tile, accumulate into acc0 / acc1.
+__device__ __forceinline__ uint32_t word_of(const uint4 &v, int i) {
+  return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+}
+
+// One stage of one warp: lane (g, t) dequantises line t of rows g and g + 8
+// (256 codes each) and multiplies with the NG token groups of the activation
+// tile, accumulating into acc0 / acc1.
 template <int NG>
-__device__ __forceinline__ void mma_chunk(const uint8_t *sw, const uint8_t *ssf, const uint4 *act,
-                                          int c, int wrow, int g, int t, bool lane_k,
+__device__ __forceinline__ void mma_stage(const uint8_t *sw, const uint8_t *ssf, const uint4 *act_c,
+                                          int g, int t, int lane, bool line_ok,
                                           float (&acc0)[kNG][4], float (&acc1)[kNG][4]) {
-  uint4 wa[2], wb[2];
-  uint32_t sfa_w = 0, sfb_w = 0;
-  if (lane_k) {
-    // 128-byte swizzle: 16-byte chunk j of row r sits at chunk j ^ (r & 7); r & 7 == g
-    const uint4 *pa = reinterpret_cast<const uint4 *>(sw + wrow * kWStride);
-    const uint4 *pb = reinterpret_cast<const uint4 *>(sw + (wrow + 8) * kWStride);
-    wa[0] = pa[(2 * t) ^ g];
-    wa[1] = pa[(2 * t + 1) ^ g];
-    wb[0] = pb[(2 * t) ^ g];
-    wb[1] = pb[(2 * t + 1) ^ g];
-    sfa_w = *reinterpret_cast<const uint32_t *>(ssf + wrow * kSFStride + 4 * t);
-    sfb_w = *reinterpret_cast<const uint32_t *>(ssf + (wrow + 8) * kSFStride + 4 * t);
-  } else {
-    wa[0] = wa[1] = wb[0] = wb[1] = make_uint4(0u, 0u, 0u, 0u);
+  const uint8_t *ra = sw + g * kRowW + t * 128;
+  const uint8_t *rb = ra + 8 * kRowW;
+  const int key = ((g & 1) << 2) | t;  // rows g and g + 8 share the parity
+  uint4 sa = make_uint4(0u, 0u, 0u, 0u), sb = sa;
+  if (line_ok) {
+    sa = *reinterpret_cast<const uint4 *>(ssf + g * kRowSF + t * 16);
+    sb = *reinterpret_cast<const uint4 *>(ssf + (g + 8) * kRowSF + t * 16);
   }
-  const uint32_t sa01 = e4m3x2_to_f16x2(sfa_w & 0xFFFFu), sa23 = e4m3x2_to_f16x2(sfa_w >> 16);
-  const uint32_t sb01 = e4m3x2_to_f16x2(sfb_w & 0xFFFFu), sb23 = e4m3x2_to_f16x2(sfb_w >> 16);
-  const uint4 *tile = act + c * NG * 256;
 #pragma unroll
-  for (int sp = 0; sp < 4; ++sp) {
-    const uint32_t sca = (sp & 1) ? bcast_hi(sp < 2 ? sa01 : sa23) : bcast_lo(sp < 2 ? sa01 : sa23);
-    const uint32_t scb = (sp & 1) ? bcast_hi(sp < 2 ? sb01 : sb23) : bcast_lo(sp < 2 ? sb01 : sb23);
-    const uint4 &va = wa[sp >> 1];
-    const uint4 &vb = wb[sp >> 1];
-    const uint32_t ca0 = (sp & 1) ? va.z : va.x, ca1 = (sp & 1) ? va.w : va.y;
-    const uint32_t cb0 = (sp & 1) ? vb.z : vb.x, cb1 = (sp & 1) ? vb.w : vb.y;
-    uint32_t A0[4], A1[4], B0[4], B1[4];
-    e2m1x8_to_f16x2(ca0, A0[0], A0[1], A0[2], A0[3]);  // row g, MMAs 0, 1
-    e2m1x8_to_f16x2(ca1, A1[0], A1[1], A1[2], A1[3]);  // row g, MMAs 2, 3
-    e2m1x8_to_f16x2(cb0, B0[0], B0[1], B0[2], B0[3]);  // row g + 8
-    e2m1x8_to_f16x2(cb1, B1[0], B1[1], B1[2], B1[3]);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      A0[q] = hmul2(A0[q], sca);
-      A1[q] = hmul2(A1[q], sca);
-      B0[q] = hmul2(B0[q], scb);
-      B1[q] = hmul2(B1[q], scb);
+  for (int q = 0; q < 8; ++q) {
+    // 16-byte chunk q of the line: 32 codes, scale bytes 2q and 2q + 1
+    uint4 wa = make_uint4(0u, 0u, 0u, 0u), wb = wa;
+    if (line_ok) {
+      wa = *reinterpret_cast<const uint4 *>(ra + ((q ^ key) << 4));
+      wb = *reinterpret_cast<const uint4 *>(rb + ((q ^ key) << 4));
     }
+    const uint32_t swa = word_of(sa, q >> 1), swb = word_of(sb, q >> 1);
+    const uint32_t pa = e4m3x2_to_f16x2((q & 1) ? (swa >> 16) : (swa & 0xFFFFu));
+    const uint32_t pb = e4m3x2_to_f16x2((q & 1) ? (swb >> 16) : (swb & 0xFFFFu));
 #pragma unroll
-    for (int G = 0; G < NG; ++G) {
-      const uint4 bh0 = tile[act_index(0, NG, G, sp, 0, g, t)];
-      const uint4 bh1 = tile[act_index(0, NG, G, sp, 1, g, t)];
-      mma_16816_f16(acc0[G], A0[0], B0[0], A0[1], B0[1], bh0.x, bh0.y);
-      mma_16816_f16(acc1[G], A1[0], B1[0], A1[1], B1[1], bh1.x, bh1.y);
-      mma_16816_f16(acc0[G], A0[2], B0[2], A0[3], B0[3], bh0.z, bh0.w);
-      mma_16816_f16(acc1[G], A1[2], B1[2], A1[3], B1[3], bh1.z, bh1.w);
+    for (int wd = 0; wd < 4; ++wd) {
+      const uint32_t sca = wd < 2 ? bcast_lo(pa) : bcast_hi(pa);
+      const uint32_t scb = wd < 2 ? bcast_lo(pb) : bcast_hi(pb);
+      uint32_t A[4], B[4];
+      e2m1x8_to_f16x2(word_of(wa, wd), A[0], A[1], A[2], A[3]);  // row g
+      e2m1x8_to_f16x2(word_of(wb, wd), B[0], B[1], B[2], B[3]);  // row g + 8
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        A[i] = hmul2(A[i], sca);
+        B[i] = hmul2(B[i], scb);
+      }
+#pragma unroll
+      for (int G = 0; G < NG; ++G) {
+        const uint4 bv = act_c[act_index(0, NG, G, 4 * q + wd, lane)];
+        mma_16816_f16(acc0[G], A[0], B[0], A[1], B[1], bv.x, bv.y);
+        mma_16816_f16(acc1[G], A[2], B[2], A[3], B[3], bv.z, bv.w);
+      }
     }
   }
 }
 
-template <int MODE, bool SF_TMA>
+template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
-    grouped_gemv_mma_kernel(const Params p, const int ts, const __grid_constant__ CUtensorMap tmap_w,
-                            const __grid_constant__ CUtensorMap tmap_sf) {
+    grouped_gemv_mma_kernel(const Params p, const int ts, const __grid_constant__ CUtensorMap tmap_w) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint4 *act = reinterpret_cast<uint4 *>(smem + kOffAct);
   uint16_t *staging = reinterpret_cast<uint16_t *>(smem + kOffStaging);
   uint32_t *prefix = reinterpret_cast<uint32_t *>(smem + kOffPrefix);
-  uint32_t *s_start = reinterpret_cast<uint32_t *>(smem + kOffStart);
-  int32_t *s_eid = reinterpret_cast<int32_t *>(smem + kOffEid);
   uint32_t *s_pair = reinterpret_cast<uint32_t *>(smem + kOffPair);
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + kOffBar);
-  uint64_t *empty = full + kStages;
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffMisc);
 
   const int warp = threadIdx.x >> 5;
@@ -157,17 +160,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int RB = (N + 15) / 16;
   const uint32_t A = p.stats[1];
 
-  for (uint32_t i = threadIdx.x; i <= A; i += blockDim.x) {
-    s_start[i] = p.start[i];
-    if (i < A) s_eid[i] = p.eids[i];
-  }
-  __syncthreads();
-  if (warp == 0) build_prefix(prefix, s_start, A, (uint32_t)ts, RB, lane);
+  if (warp == 0) build_prefix(prefix, p.start, A, (uint32_t)ts, RB, lane);
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full[s], SF_TMA ? 1u : 33u);
-      mbar_init(&empty[s], (uint32_t)kCW);
-    }
+    // one arrival with the TMA byte count + one cp.async arrival per lane
+    for (int i = 0; i < kCW * kSlots; ++i) mbar_init(&full[i], 33u);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -177,84 +173,84 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t u_begin = (uint32_t)(((uint64_t)U * blockIdx.x) / gridDim.x);
   const uint32_t u_end = (uint32_t)(((uint64_t)U * (blockIdx.x + 1)) / gridDim.x);
   if (u_begin >= u_end) return;
-  const int nchunks = (K + kKC - 1) / kKC;
+  const int nst = (K + kKS - 1) / kKS;  // stages per block
+  const int lines_total = K / 256;
   const int64_t sf_row_bytes = K / 16;
-  const Meta meta{prefix, s_start, s_eid, N};
+  const Meta meta{prefix, p.start, p.eids, N};
+  uint8_t *wring = smem + kOffW + (size_t)warp * kSlots * kStageW;
+  uint8_t *sring = smem + kOffSF + (size_t)warp * kSlots * kStageSF;
+  uint64_t *wfull = full + warp * kSlots;
+  const uint64_t policy = l2_evict_first_policy();
+  if (lane == 0) prefetch_tmap(&tmap_w);
 
-  auto wait = [&](uint64_t *bar, uint32_t parity) {
-    if (*abort_flag) return;
-    if (!mbar_wait_bounded(bar, parity, kWaitLimitNs)) *abort_flag = 1;
-  };
-
-  if (warp == kCW) {
-    // ================================================================ TMA producer
-    RoundIter iter{u_begin, u_end, 0, (uint32_t)ts};
-    Round r;
-    uint32_t it = 0;
-    const uint64_t policy = l2_evict_first_policy();
-    if (lane == 0) {
-      prefetch_tmap(&tmap_w);
-      if (SF_TMA) prefetch_tmap(&tmap_sf);
-    }
-    while (iter.next(meta, RB, r)) {
-      for (int c = 0; c < nchunks; ++c, ++it) {
-        const int s = (int)(it % kStages);
-        wait(&empty[s], ((it / kStages) & 1u) ^ 1u);
-        if (*abort_flag) continue;
-        const int k0 = c * kKC;
-        uint8_t *sw = smem + (size_t)s * kStageBytes;
-        uint8_t *ssf = sw + kStageW;
-        if (lane == 0)
-          mbar_arrive_expect_tx(&full[s], (uint32_t)r.nblk * (kBoxW + (SF_TMA ? kBoxSF : 0)));
-        __syncwarp();
-        if (lane < r.nblk) {
-          tma_load_3d(sw + lane * kBoxW, &tmap_w, k0 / 2, r.n0 + 16 * lane, r.e, &full[s], policy);
-          if (SF_TMA)
-            tma_load_3d(ssf + lane * kBoxSF, &tmap_sf, k0 / 16, r.n0 + 16 * lane, r.e, &full[s],
-                        policy);
-        }
-        if (!SF_TMA) {
-          const uint32_t sb = (uint32_t)min(kKC, K - k0) / 16;
-          const uint8_t *sbase = p.sfw + ((int64_t)r.e * N + r.n0) * sf_row_bytes + k0 / 16;
-          for (int row = lane; row < r.nrows; row += 32)
-            for (uint32_t q = 0; q < sb; q += 4)
-              cp_async4(ssf + row * kSFStride + q, sbase + row * sf_row_bytes + q);
-          cp_async_mbar_arrive_noinc(&full[s]);
-        }
+  // ---- producer side of this warp's pipeline: the next (round, stage) of its blocks
+  RoundIter piter{u_begin, u_end, 0, (uint32_t)ts, (uint32_t)kCW};
+  Round pr;
+  int pc = 0;
+  bool pvalid = false;
+  auto next_own_round = [&]() {
+    pvalid = false;
+    pc = 0;
+    while (piter.next(meta, RB, pr))
+      if (warp < pr.nblk) {
+        pvalid = true;
+        break;
       }
+  };
+  next_own_round();
+  uint32_t produced = 0;
+  auto produce = [&]() {
+    // lane 0's view of the abort flag decides for the whole warp
+    if (!pvalid || __shfl_sync(0xFFFFFFFFu, *abort_flag, 0)) return;
+    const int slot = (int)(produced % kSlots);
+    uint8_t *sw = wring + slot * kStageW;
+    uint8_t *ssf = sring + slot * kStageSF;
+    uint64_t *bar = &wfull[slot];
+    const int n0 = pr.n0 + 16 * warp;
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar, (uint32_t)kStageW);
+      tma_load_4d(sw, &tmap_w, 0, pc * kLines, n0, pr.e, bar, policy);
     }
-    return;
-  }
+    for (int piece = lane; piece < 16 * kLines; piece += 32) {
+      const int r = piece / kLines, j = piece % kLines;
+      const int line = pc * kLines + j;
+      if (n0 + r < N && line < lines_total)
+        cp_async16(ssf + r * kRowSF + j * 16,
+                   p.sfw + ((int64_t)pr.e * N + n0 + r) * sf_row_bytes + line * 16);
+    }
+    cp_async_mbar_arrive_noinc(bar);
+    ++produced;
+    if (++pc == nst) next_own_round();
+  };
+  for (int s = 0; s < kSlots; ++s) produce();
 
-  // ================================================================== compute warps
-  const int cw = warp;
+  // ---- consumer side
   const int g = lane >> 2, t = lane & 3;
-  const int wrow = cw * 16 + g;  // round-local row of a0 (a1: wrow + 8)
-  RoundIter iter{u_begin, u_end, 0, (uint32_t)ts};
+  RoundIter iter{u_begin, u_end, 0, (uint32_t)ts, (uint32_t)kCW};
   Round r;
-  uint32_t it = 0;
+  uint32_t consumed = 0;
   uint32_t pass_key = 0xFFFFFFFFu;
   int ng = 0;
-  const int kpad = nchunks * kKC;
+  const int kpad = nst * kKS;
 
   while (iter.next(meta, RB, r)) {
     if (r.tok0 != pass_key) {
       // ---- new (expert, pass): build its fp16 activation tile for the whole K
-      named_bar_sync(1, kCW * 32);  // every warp is done with the previous tile
+      named_bar_sync(1, kThreads);  // every warp is done with the previous tile
       ng = (r.ntok + 7) / 8;
-      for (int i = threadIdx.x; i < r.ntok; i += kCW * 32) s_pair[i] = p.order[r.tok0 + i];
-      named_bar_sync(1, kCW * 32);
+      for (int i = threadIdx.x; i < r.ntok; i += kThreads) s_pair[i] = p.order[r.tok0 + i];
+      named_bar_sync(1, kThreads);
       unsigned range_bad = 0;
       const int per_tok = kpad / 8;  // 8-column slices per token
       const int ntask = r.ntok * per_tok;
       // each thread converts up to kBatch slices per step with all loads issued first
-      constexpr int kBatch = 8;
-      for (int base = 0; base < ntask; base += kCW * 32 * kBatch) {
+      constexpr int kBatch = 4;
+      for (int base = 0; base < ntask; base += kThreads * kBatch) {
         uint4 v[kBatch];
         uint32_t sv[kBatch];
 #pragma unroll
         for (int b = 0; b < kBatch; ++b) {
-          const int task = base + b * kCW * 32 + threadIdx.x;
+          const int task = base + b * kThreads + threadIdx.x;
           v[b] = make_uint4(0u, 0u, 0u, 0u);
           sv[b] = 0u;
           if (task < ntask) {
@@ -274,7 +270,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
 #pragma unroll
         for (int b = 0; b < kBatch; ++b) {
-          const int task = base + b * kCW * 32 + threadIdx.x;
+          const int task = base + b * kThreads + threadIdx.x;
           if (task >= ntask) continue;
           const int tau = task / per_tok;
           const int k = (task % per_tok) * 8;
@@ -302,52 +298,55 @@ __global__ void __launch_bounds__(kThreads, 1)
               hv.w = hmul2(q3, sc);
             }
           }
-          // fragment slot of columns [k, k + 8) of token tau
-          const int c = k / kKC, kk = k % kKC, L = kk / 8;
-          act[act_index(c, ng, tau / 8, (L & 7) >> 1, L & 1, tau & 7, L >> 3)] = hv;
+          // columns [k, k + 8): stage c, line lt, MMA pair m of lane (tau % 8, lt)
+          const int c = k / kKS, kk = k % kKS, lt = kk / 256, m = (kk % 256) / 8;
+          act[act_index(c, ng, tau / 8, m, (tau & 7) * 4 + lt)] = hv;
         }
       }
       if (MODE == MOE_W4A16 && range_bad) raise_device_error(MOE_DEVERR_ACT_RANGE);
-      named_bar_sync(1, kCW * 32);
+      named_bar_sync(1, kThreads);
       pass_key = r.tok0;
     }
 
-    const bool has_rows = cw < r.nblk;
+    if (warp >= r.nblk) continue;
     float acc0[kNG][4], acc1[kNG][4];
 #pragma unroll
     for (int G = 0; G < kNG; ++G)
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc0[G][i] = acc1[G][i] = 0.f;
 
-    for (int c = 0; c < nchunks; ++c, ++it) {
-      const int s = (int)(it % kStages);
-      wait(&full[s], (it / kStages) & 1u);
-      if (has_rows && !*abort_flag) {
-        const uint8_t *sw = smem + (size_t)s * kStageBytes;
-        const uint8_t *ssf = sw + kStageW;
-        const bool lane_k = 64 * t < min(kKC, K - c * kKC);
-        switch (ng) {
-          case 1: mma_chunk<1>(sw, ssf, act, c, wrow, g, t, lane_k, acc0, acc1); break;
-          case 2: mma_chunk<2>(sw, ssf, act, c, wrow, g, t, lane_k, acc0, acc1); break;
-          case 3: mma_chunk<3>(sw, ssf, act, c, wrow, g, t, lane_k, acc0, acc1); break;
-          default: mma_chunk<4>(sw, ssf, act, c, wrow, g, t, lane_k, acc0, acc1); break;
-        }
+    for (int c = 0; c < nst; ++c) {
+      const int slot = (int)(consumed % kSlots);
+      if (!*abort_flag &&
+          !mbar_wait_bounded(&wfull[slot], (consumed / kSlots) & 1u, kWaitLimitNs))
+        *abort_flag = 1;
+      if (!*abort_flag) {
+        const uint8_t *sw = wring + slot * kStageW;
+        const uint8_t *ssf = sring + slot * kStageSF;
+        const bool line_ok = c * kLines + t < lines_total;
+        const uint4 *act_c = act + act_index(c, ng, 0, 0, 0);
+        if (ng == 1)
+          mma_stage<1>(sw, ssf, act_c, g, t, lane, line_ok, acc0, acc1);
+        else
+          mma_stage<2>(sw, ssf, act_c, g, t, lane, line_ok, acc0, acc1);
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
+      ++consumed;
+      __syncwarp();  // every lane is done with the slot before it is refilled
+      produce();
     }
 
-    // ---- round epilogue: scale, round to bf16, transpose, 16-byte stores
-    if (has_rows && !*abort_flag) {
+    // ---- block epilogue: scale, round to bf16, transpose, 16-byte stores
+    if (!*abort_flag) {
       const float gw = p.w_global ? p.w_global[r.e] : 1.0f;
       const float f = __fmul_rn(gw, p.g_a);
-      uint16_t *st = staging + cw * (kMaxTS * 16);
+      uint16_t *st = staging + warp * (kMaxTS * 16);
+      auto y = [&](int G, int i) { return __fmul_rn(acc0[G][i] + acc1[G][i], f); };
 #pragma unroll
       for (int G = 0; G < kNG; ++G) {
         if (G < ng) {
           const int c0 = G * 8 + 2 * t;
-          const uint32_t lo = pack_bf16x2((acc0[G][0] + acc1[G][0]) * f, (acc0[G][1] + acc1[G][1]) * f);
-          const uint32_t hi = pack_bf16x2((acc0[G][2] + acc1[G][2]) * f, (acc0[G][3] + acc1[G][3]) * f);
+          const uint32_t lo = pack_bf16x2(y(G, 0), y(G, 1));
+          const uint32_t hi = pack_bf16x2(y(G, 2), y(G, 3));
           st[c0 * 16 + g] = (uint16_t)(lo & 0xFFFFu);
           st[(c0 + 1) * 16 + g] = (uint16_t)(lo >> 16);
           st[c0 * 16 + g + 8] = (uint16_t)(hi & 0xFFFFu);
@@ -355,7 +354,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       __syncwarp();
-      const int nw = r.n0 + cw * 16;
+      const int nw = r.n0 + warp * 16;
       for (int task = lane; task < r.ntok * 2; task += 32) {
         const int col = task >> 1, half = task & 1;
         const int n = nw + half * 8;
@@ -366,6 +365,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       __syncwarp();
+    }
+  }
+
+  // After a timed-out wait, let this warp's copies still in flight land
+  // before the CTA exits (bounded again).
+  if (*abort_flag && lane == 0) {
+    for (int s = 0; s < kSlots; ++s) {
+      const uint32_t uses =
+          produced > (uint32_t)s ? (produced - (uint32_t)s + kSlots - 1) / kSlots : 0u;
+      if (uses) mbar_wait_bounded(&wfull[s], (uses - 1) & 1u, kDrainLimitNs);
     }
   }
 }

@@ -117,13 +117,30 @@ bool encode_u8_3d(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 4-D uint32 map over the codes of [E][N][K/2] seen as [E][N][K/256 lines]
+// [32 words of a 128-byte line]; box = 16 rows x `lines` lines, 128-byte
+// swizzle.  Needs K % 256 == 0.
+bool encode_lines_4d(CUtensorMap *m, const void *base, uint64_t K, uint64_t N, uint64_t E,
+                     uint32_t lines) {
+  auto fn = tensor_map_encoder();
+  if (!fn) return false;
+  const cuuint64_t dims[4] = {32, K / 256, N, E};
+  const cuuint64_t strides[3] = {128, K / 2, (K / 2) * N};
+  const cuuint32_t box[4] = {32, lines, 16, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, const_cast<void *>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Descriptors of the expert library, cached by (pointers, shape): encoding
 // costs a driver call, and graph replays reuse the captured parameters anyway.
 struct LibMaps {
   const void *w = nullptr, *sfw = nullptr;
   int E = 0, N = 0, K = 0;
-  bool sf_tma = false;
-  CUtensorMap tw, tsf;
+  bool sf_tma = false;  // K % 256 == 0: scale boxes for the tensor-memory variant,
+                        // and the line map of the decode variant
+  CUtensorMap tw, tsf, tlines;
 };
 constexpr int kMapCache = 8;
 LibMaps g_maps[kMapCache];
@@ -145,14 +162,17 @@ bool library_maps(const uint8_t *w, const uint8_t *sfw, int E, int N, int K, Lib
   m.K = K;
   m.sf_tma = (K % 256) == 0;
   std::memset(&m.tsf, 0, sizeof m.tsf);
-  // both GEMV variants read 16-row x 128-byte weight boxes and 16-row x 16-byte scale boxes
-  static_assert(moe::gemv::tc::kWStride == 128 && moe::gemv::mma::kWStride == 128, "box width");
-  static_assert(moe::gemv::tc::kSFStride == 16 && moe::gemv::mma::kSFStride == 16, "box width");
+  std::memset(&m.tlines, 0, sizeof m.tlines);
+  // the tensor-memory variant reads 16-row x 128-byte weight boxes and 16-row x 16-byte scale boxes
+  static_assert(moe::gemv::tc::kWStride == 128 && moe::gemv::tc::kSFStride == 16, "box width");
   if (!encode_u8_3d(&m.tw, w, (uint64_t)K / 2, (uint64_t)N, (uint64_t)E, 128, 16,
                     CU_TENSOR_MAP_SWIZZLE_128B))
     return false;
   if (m.sf_tma && !encode_u8_3d(&m.tsf, sfw, (uint64_t)K / 16, (uint64_t)N, (uint64_t)E, 16, 16,
                                 CU_TENSOR_MAP_SWIZZLE_NONE))
+    return false;
+  if (m.sf_tma && !encode_lines_4d(&m.tlines, w, (uint64_t)K, (uint64_t)N, (uint64_t)E,
+                                   (uint32_t)moe::gemv::mma::kLines))
     return false;
   g_maps[g_maps_next] = m;
   g_maps_next = (g_maps_next + 1) % kMapCache;
@@ -282,12 +302,23 @@ moe_status_t moe_dispatch_mxfp4(const void *input_tokens, int32_t N, int32_t K, 
   int sms = 0;
   moe_status_t st = check_device(&sms);
   if (st != MOE_OK) return st;
+  // segments of 256 columns per warp task: the largest of 8, 4, 2, 1 that
+  // still gives every SM about 8 warps
   const int wpb = moe::disp::kWarpsPerBlock;
-  const int64_t groups = ((K + 255) / 256 + moe::disp::kSegGroup - 1) / moe::disp::kSegGroup;
+  const int64_t segs = (K + 255) / 256;
+  int seg = 8;
+  while (seg > 1 && (int64_t)N * ((segs + seg - 1) / seg) < (int64_t)sms * 8) seg /= 2;
+  const int64_t groups = (segs + seg - 1) / seg;
   int64_t blocks = ((int64_t)N * groups + wpb - 1) / wpb;
   if (blocks < 1) blocks = 1;
   if (blocks > (int64_t)sms * 16) blocks = (int64_t)sms * 16;
-  moe::disp::dispatch_mxfp4_kernel<<<(unsigned)blocks, wpb * 32, 0, s>>>(
+  void (*kern)(const uint16_t *, int32_t, int32_t, int32_t, int32_t, const uint32_t *,
+               const uint32_t *, const int32_t *, const uint32_t *, uint8_t *, int64_t, int32_t,
+               uint32_t *) = seg == 8   ? moe::disp::dispatch_mxfp4_kernel<8>
+                             : seg == 4 ? moe::disp::dispatch_mxfp4_kernel<4>
+                             : seg == 2 ? moe::disp::dispatch_mxfp4_kernel<2>
+                                        : moe::disp::dispatch_mxfp4_kernel<1>;
+  kern<<<(unsigned)blocks, wpb * 32, 0, s>>>(
       static_cast<const uint16_t *>(input_tokens), N, K, top_k, E, restore_token_order,
       expert_start_indices, expert_ids, expert_usage_stats, recv_buf, recv_capacity,
       (int32_t)moe_mxfp4_row_stride(K), recv_counts);
@@ -388,26 +419,23 @@ moe_status_t moe_grouped_gemv_nvfp4(moe_gemv_mode_t mode, const void *act, const
   p.out = static_cast<uint16_t *>(out);
   LibMaps maps;
   if (!library_maps(w, sfw, E, N, K, &maps)) return MOE_ERR_CUDA;
-  // Decode-sized passes (few tokens per expert on average) take the register-
-  // dequant mma.sync variant; many tokens per expert take the tensor-memory
-  // variant, whose tcgen05 MMA has a fixed per-instruction cost up to N = 64.
-  const int ts_mma = mma::tokens_per_pass(K);
-  bool use_mma = ts_mma >= 8 && (S / E) < 48;
+  // Decode-sized passes (no more tokens per expert on average than one pass
+  // of the register-dequant mma.sync variant holds) take that variant; more
+  // tokens per expert take the tensor-memory variant, whose tcgen05 MMA has a
+  // fixed per-instruction cost up to N = 64 and whose passes hold 64 tokens.
+  const int ts_mma = maps.sf_tma ? mma::tokens_per_pass(K) : 0;
+  bool use_mma = ts_mma >= 8 && S <= (int64_t)ts_mma * E;
   // test hook: MOE_GEMV_VARIANT=mma|tc forces a variant (both are exact for every input)
   if (const char *v = std::getenv("MOE_GEMV_VARIANT")) {
     if (v[0] == 'm' && ts_mma >= 8) use_mma = true;
     if (v[0] == 't') use_mma = false;
   }
   if (use_mma) {
-    void (*kern)(const Params, const int, const CUtensorMap, const CUtensorMap);
-    if (mode == MOE_W4A16)
-      kern = maps.sf_tma ? mma::grouped_gemv_mma_kernel<MOE_W4A16, true>
-                         : mma::grouped_gemv_mma_kernel<MOE_W4A16, false>;
-    else
-      kern = maps.sf_tma ? mma::grouped_gemv_mma_kernel<MOE_W4A4, true>
-                         : mma::grouped_gemv_mma_kernel<MOE_W4A4, false>;
+    void (*kern)(const Params, const int, const CUtensorMap) =
+        mode == MOE_W4A16 ? mma::grouped_gemv_mma_kernel<MOE_W4A16>
+                          : mma::grouped_gemv_mma_kernel<MOE_W4A4>;
     if ((st = set_smem(kern, mma::kSmemBytes)) != MOE_OK) return st;
-    kern<<<(unsigned)sms, mma::kThreads, mma::kSmemBytes, s>>>(p, ts_mma, maps.tw, maps.tsf);
+    kern<<<(unsigned)sms, mma::kThreads, mma::kSmemBytes, s>>>(p, ts_mma, maps.tlines);
     return launch_status();
   }
   void (*kern)(const Params, const CUtensorMap, const CUtensorMap);

@@ -226,6 +226,15 @@ GEMV_CASES = [
                                     N_out=264), "w4a4"),
     # minimal K, N
     ("minimal", wl.small_config("minimal", N=3, real=3, K=64, E=2, top_k=1, N_out=8), "w4a16"),
+    # K % 256 == 0 with a partial last stage of 1024 columns (2304 = 2 x 1024 + 256),
+    # ragged row block, 8-token passes and two-group passes of the decode variant
+    ("lines-w4a16", wl.small_config("lines", N=40, real=37, K=2304, E=5, top_k=2, N_out=200),
+     "w4a16"),
+    ("lines-w4a4", wl.small_config("lines", N=40, real=37, K=2304, E=5, top_k=2, N_out=200),
+     "w4a4"),
+    # decode-like: K = 2048 (two full stages), about 16 tokens per expert
+    ("decode-like", wl.small_config("dlike", N=64, real=64, K=2048, E=16, top_k=4, N_out=136),
+     "w4a16"),
     # activations spanning many binades (per-chunk power-of-two scaling)
     ("wide-range", wl.small_config("wide", N=24, real=24, K=1024, E=6, top_k=2, N_out=128,
                                    outlier_frac=0.05, outlier_mult=3000.0), "w4a16"),
