@@ -45,6 +45,18 @@ struct Meta {
   int N;
 };
 
+// Active expert holding unit u: the a with prefix[a] <= u < prefix[a + 1]
+// (binary search; u < prefix[A]).
+__device__ __forceinline__ int expert_of_unit(const uint32_t *prefix, uint32_t A, uint32_t u) {
+  int lo = 0, hi = (int)A - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (prefix[mid] <= u) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
+
 // Walks a CTA's unit range round by round; identical in every thread.
 struct RoundIter {
   uint32_t u, u_end;
@@ -72,6 +84,42 @@ struct RoundIter {
     return true;
   }
 };
+
+// This CTA's share [u0, u1) of the U units, cut at round boundaries: every
+// pass (RB units) splits into ceil(RB / rbk) rounds of up to rbk blocks, and
+// the grid shares the rounds evenly, so no round is split between CTAs and a
+// CTA's warps never face a partial round in the middle of a pass.
+__device__ __forceinline__ void cta_round_range(uint32_t U, int RB, int rbk, uint32_t &u0,
+                                                uint32_t &u1) {
+  const uint64_t R = (uint64_t)((RB + rbk - 1) / rbk);
+  const uint64_t T = (uint64_t)(U / (uint32_t)RB) * R;
+  const uint64_t r0 = T * blockIdx.x / gridDim.x, r1 = T * (blockIdx.x + 1) / gridDim.x;
+  u0 = (uint32_t)((r0 / R) * (uint64_t)RB + (r0 % R) * (uint64_t)rbk);
+  u1 = (uint32_t)((r1 / R) * (uint64_t)RB + (r1 % R) * (uint64_t)rbk);
+}
+
+// As cta_round_range, but when the passes (U / RB of them) are no more than
+// the CTAs, every CTA takes part of exactly one pass: pass p gets the CTAs b
+// with floor(b * P / G) == p and splits its rounds evenly among them.  Each
+// CTA then builds one activation tile and never waits for its warps between
+// passes.
+__device__ __forceinline__ void cta_pass_range(uint32_t U, int RB, int rbk, uint32_t &u0,
+                                               uint32_t &u1) {
+  const uint64_t P = U / (uint32_t)RB, G = gridDim.x, b = blockIdx.x;
+  if (P == 0 || P > G) {
+    cta_round_range(U, RB, rbk, u0, u1);
+    return;
+  }
+  const uint64_t pass = b * P / G;
+  const uint64_t first = (pass * G + P - 1) / P;        // first CTA of the pass
+  const uint64_t count = ((pass + 1) * G + P - 1) / P - first;
+  const uint64_t i = b - first;
+  const uint64_t R = (uint64_t)((RB + rbk - 1) / rbk);
+  const uint64_t r0 = R * i / count, r1 = R * (i + 1) / count;
+  const uint64_t base = pass * (uint64_t)RB;
+  u0 = (uint32_t)(base + min((uint64_t)RB, r0 * (uint64_t)rbk));
+  u1 = (uint32_t)(base + min((uint64_t)RB, r1 * (uint64_t)rbk));
+}
 
 __device__ __forceinline__ uint32_t bcast_lo(uint32_t h) { return __byte_perm(h, h, 0x1010); }
 __device__ __forceinline__ uint32_t bcast_hi(uint32_t h) { return __byte_perm(h, h, 0x3232); }

@@ -60,13 +60,19 @@ constexpr int kGroupStageBytes = 8 * kKS * 2;  // fp16 tile of one 8-token group
 constexpr int kActBytes = 64 * 1024;
 constexpr int kStagingBytes = kCW * kMaxTS * 16 * 2;
 constexpr uint64_t kDrainLimitNs = 100000000ull;  // 100 ms
+// 16-byte activation slices per thread in a pass setup: the tile holds
+// kActBytes / 16 slices, spread over the CTA.
+constexpr int kSetupTasks = kActBytes / 16 / kThreads;
 
 constexpr size_t kOffW = 0;
 constexpr size_t kOffSF = kOffW + (size_t)kCW * kSlots * kStageW;
 constexpr size_t kOffAct = kOffSF + (size_t)kCW * kSlots * kStageSF;
 constexpr size_t kOffStaging = kOffAct + kActBytes;
+constexpr int kMaxActive = 512;              // active experts this variant takes
 constexpr size_t kOffPrefix = kOffStaging + kStagingBytes;
-constexpr size_t kOffPair = kOffPrefix + (kMaxExperts + 4) * 4;
+constexpr size_t kOffStart = kOffPrefix + (kMaxActive + 4) * 4;
+constexpr size_t kOffEid = kOffStart + (kMaxActive + 4) * 4;
+constexpr size_t kOffPair = kOffEid + (kMaxActive + 4) * 4;
 constexpr size_t kOffBar = kOffPair + kMaxTS * 4;
 constexpr size_t kOffMisc = kOffBar + (size_t)kCW * kSlots * 8;
 constexpr size_t kSmemBytes = kOffMisc + 16 + 1024;
@@ -141,6 +147,51 @@ __device__ __forceinline__ void mma_stage(const uint8_t *sw, const uint8_t *ssf,
   }
 }
 
+// Walks the rounds of a CTA's range [u, u_end) (round-aligned) in order: the
+// first block of the round steps by kCW within a pass, then the pass, then
+// the active expert, so only the starting position needs a division.
+struct RoundWalk {
+  uint32_t u, u_end;
+  int a;
+  uint32_t pass;
+  int rb;
+  __device__ __forceinline__ void init(const Meta &m, uint32_t A, int RB, uint32_t u0,
+                                       uint32_t u1) {
+    u = u0;
+    u_end = u1;
+    a = expert_of_unit(m.prefix, A, u0);
+    const uint32_t v = u0 - m.prefix[a];
+    pass = v / (uint32_t)RB;
+    rb = (int)(v % (uint32_t)RB);
+  }
+  __device__ __forceinline__ bool next(const Meta &m, int RB, uint32_t ts, Round &r) {
+    if (u >= u_end) return false;
+    const uint32_t s0 = m.start[a], c = m.start[a + 1] - s0;
+    const uint32_t first = pass * ts;
+    int nblk = RB - rb;
+    if (nblk > kCW) nblk = kCW;
+    if ((uint32_t)nblk > u_end - u) nblk = (int)(u_end - u);
+    r.e = m.eid[a];
+    r.tok0 = s0 + first;
+    r.ntok = (int)min(ts, c - first);
+    r.n0 = rb * 16;
+    r.nrows = min(nblk * 16, m.N - r.n0);
+    r.nblk = nblk;
+    u += (uint32_t)nblk;
+    rb += nblk;
+    if (rb == RB) {
+      rb = 0;
+      if (first + ts >= c) {
+        ++a;
+        pass = 0;
+      } else {
+        ++pass;
+      }
+    }
+    return true;
+  }
+};
+
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemv_mma_kernel(const Params p, const int ts, const __grid_constant__ CUtensorMap tmap_w) {
@@ -150,6 +201,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint4 *act = reinterpret_cast<uint4 *>(smem + kOffAct);
   uint16_t *staging = reinterpret_cast<uint16_t *>(smem + kOffStaging);
   uint32_t *prefix = reinterpret_cast<uint32_t *>(smem + kOffPrefix);
+  uint32_t *s_start = reinterpret_cast<uint32_t *>(smem + kOffStart);
+  int32_t *s_eid = reinterpret_cast<int32_t *>(smem + kOffEid);
   uint32_t *s_pair = reinterpret_cast<uint32_t *>(smem + kOffPair);
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + kOffBar);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffMisc);
@@ -160,7 +213,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int RB = (N + 15) / 16;
   const uint32_t A = p.stats[1];
 
-  if (warp == 0) build_prefix(prefix, p.start, A, (uint32_t)ts, RB, lane);
+  // the grouping of the active experts (at most kMaxActive, checked on the host)
+  // stays in shared memory: every round looks it up
+  for (uint32_t i = threadIdx.x; i <= A; i += blockDim.x) {
+    s_start[i] = p.start[i];
+    if (i < A) s_eid[i] = p.eids[i];
+  }
+  __syncthreads();
+  if (warp == 0) build_prefix(prefix, s_start, A, (uint32_t)ts, RB, lane);
   if (threadIdx.x == 0) {
     // one arrival with the TMA byte count + one cp.async arrival per lane
     for (int i = 0; i < kCW * kSlots; ++i) mbar_init(&full[i], 33u);
@@ -169,14 +229,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   __syncthreads();
 
-  const uint32_t U = prefix[A];
-  const uint32_t u_begin = (uint32_t)(((uint64_t)U * blockIdx.x) / gridDim.x);
-  const uint32_t u_end = (uint32_t)(((uint64_t)U * (blockIdx.x + 1)) / gridDim.x);
+  uint32_t u_begin, u_end;
+  cta_pass_range(prefix[A], RB, kCW, u_begin, u_end);
   if (u_begin >= u_end) return;
   const int nst = (K + kKS - 1) / kKS;  // stages per block
   const int lines_total = K / 256;
   const int64_t sf_row_bytes = K / 16;
-  const Meta meta{prefix, p.start, p.eids, N};
+  const Meta meta{prefix, s_start, s_eid, N};
   uint8_t *wring = smem + kOffW + (size_t)warp * kSlots * kStageW;
   uint8_t *sring = smem + kOffSF + (size_t)warp * kSlots * kStageSF;
   uint64_t *wfull = full + warp * kSlots;
@@ -184,14 +243,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (lane == 0) prefetch_tmap(&tmap_w);
 
   // ---- producer side of this warp's pipeline: the next (round, stage) of its blocks
-  RoundIter piter{u_begin, u_end, 0, (uint32_t)ts, (uint32_t)kCW};
+  RoundWalk piter;
+  piter.init(meta, A, RB, u_begin, u_end);
   Round pr;
   int pc = 0;
   bool pvalid = false;
   auto next_own_round = [&]() {
     pvalid = false;
     pc = 0;
-    while (piter.next(meta, RB, pr))
+    while (piter.next(meta, RB, (uint32_t)ts, pr))
       if (warp < pr.nblk) {
         pvalid = true;
         break;
@@ -226,82 +286,82 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // ---- consumer side
   const int g = lane >> 2, t = lane & 3;
-  RoundIter iter{u_begin, u_end, 0, (uint32_t)ts, (uint32_t)kCW};
+  RoundWalk iter;
+  iter.init(meta, A, RB, u_begin, u_end);
   Round r;
   uint32_t consumed = 0;
   uint32_t pass_key = 0xFFFFFFFFu;
   int ng = 0;
   const int kpad = nst * kKS;
 
-  while (iter.next(meta, RB, r)) {
+  while (iter.next(meta, RB, (uint32_t)ts, r)) {
     if (r.tok0 != pass_key) {
-      // ---- new (expert, pass): build its fp16 activation tile for the whole K
-      named_bar_sync(1, kThreads);  // every warp is done with the previous tile
-      ng = (r.ntok + 7) / 8;
-      for (int i = threadIdx.x; i < r.ntok; i += kThreads) s_pair[i] = p.order[r.tok0 + i];
-      named_bar_sync(1, kThreads);
-      unsigned range_bad = 0;
+      // ---- new (expert, pass): build its fp16 activation tile for the whole K.
+      // The loads (token order, then activation slices) are issued before the
+      // barrier that frees the previous tile, so their latency overlaps it.
       const int per_tok = kpad / 8;  // 8-column slices per token
-      const int ntask = r.ntok * per_tok;
-      // each thread converts up to kBatch slices per step with all loads issued first
-      constexpr int kBatch = 4;
-      for (int base = 0; base < ntask; base += kThreads * kBatch) {
-        uint4 v[kBatch];
-        uint32_t sv[kBatch];
+      const int ntask = r.ntok * per_tok;  // at most kSetupTasks * kThreads
+      uint4 v[kSetupTasks];
+      uint32_t sv[kSetupTasks];
+      uint32_t my_pair = 0;
+      if ((int)threadIdx.x < r.ntok) my_pair = __ldg(p.order + r.tok0 + threadIdx.x);
 #pragma unroll
-        for (int b = 0; b < kBatch; ++b) {
-          const int task = base + b * kThreads + threadIdx.x;
-          v[b] = make_uint4(0u, 0u, 0u, 0u);
-          sv[b] = 0u;
-          if (task < ntask) {
-            const int tau = task / per_tok;
-            const int k = (task % per_tok) * 8;
-            const int64_t m = (int64_t)(s_pair[tau] / (uint32_t)p.top_k);
-            if (k < K) {
-              if (MODE == MOE_W4A16) {
-                v[b] = ldg_nc_v4(static_cast<const uint16_t *>(p.act) + m * K + k);
-              } else {
-                const uint8_t *qp = static_cast<const uint8_t *>(p.act) + m * (K / 2);
-                v[b].x = __ldg(reinterpret_cast<const uint32_t *>(qp + k / 2));
-                sv[b] = p.sfa[m * (K / 16) + k / 16];
-              }
-            }
-          }
-        }
-#pragma unroll
-        for (int b = 0; b < kBatch; ++b) {
-          const int task = base + b * kThreads + threadIdx.x;
-          if (task >= ntask) continue;
+      for (int b = 0; b < kSetupTasks; ++b) {
+        const int task = b * kThreads + (int)threadIdx.x;
+        v[b] = make_uint4(0u, 0u, 0u, 0u);
+        sv[b] = 0u;
+        if (task < ntask) {
           const int tau = task / per_tok;
           const int k = (task % per_tok) * 8;
-          uint4 hv = make_uint4(0u, 0u, 0u, 0u);
+          const int64_t m = (int64_t)(__ldg(p.order + r.tok0 + tau) / (uint32_t)p.top_k);
           if (k < K) {
             if (MODE == MOE_W4A16) {
-              float f[8];
-              f[0] = bf16_lo(v[b].x); f[1] = bf16_hi(v[b].x);
-              f[2] = bf16_lo(v[b].y); f[3] = bf16_hi(v[b].y);
-              f[4] = bf16_lo(v[b].z); f[5] = bf16_hi(v[b].z);
-              f[6] = bf16_lo(v[b].w); f[7] = bf16_hi(v[b].w);
-#pragma unroll
-              for (int e = 0; e < 8; ++e) range_bad |= (fabsf(f[e]) > 65504.0f) ? 1u : 0u;
-              hv.x = pack_f16x2(f[0], f[1]);
-              hv.y = pack_f16x2(f[2], f[3]);
-              hv.z = pack_f16x2(f[4], f[5]);
-              hv.w = pack_f16x2(f[6], f[7]);
+              v[b] = ldg_nc_v4(static_cast<const uint16_t *>(p.act) + m * K + k);
             } else {
-              const uint32_t sc = bcast_lo(e4m3x2_to_f16x2(sv[b]));
-              uint32_t q0, q1, q2, q3;
-              e2m1x8_to_f16x2(v[b].x, q0, q1, q2, q3);
-              hv.x = hmul2(q0, sc);
-              hv.y = hmul2(q1, sc);
-              hv.z = hmul2(q2, sc);
-              hv.w = hmul2(q3, sc);
+              const uint8_t *qp = static_cast<const uint8_t *>(p.act) + m * (K / 2);
+              v[b].x = __ldg(reinterpret_cast<const uint32_t *>(qp + k / 2));
+              sv[b] = p.sfa[m * (K / 16) + k / 16];
             }
           }
-          // columns [k, k + 8): stage c, line lt, MMA pair m of lane (tau % 8, lt)
-          const int c = k / kKS, kk = k % kKS, lt = kk / 256, m = (kk % 256) / 8;
-          act[act_index(c, ng, tau / 8, m, (tau & 7) * 4 + lt)] = hv;
         }
+      }
+      named_bar_sync(1, kThreads);  // every warp is done with the previous tile
+      ng = (r.ntok + 7) / 8;
+      if ((int)threadIdx.x < r.ntok) s_pair[threadIdx.x] = my_pair;
+      unsigned range_bad = 0;
+#pragma unroll
+      for (int b = 0; b < kSetupTasks; ++b) {
+        const int task = b * kThreads + (int)threadIdx.x;
+        if (task >= ntask) continue;
+        const int tau = task / per_tok;
+        const int k = (task % per_tok) * 8;
+        uint4 hv = make_uint4(0u, 0u, 0u, 0u);
+        if (k < K) {
+          if (MODE == MOE_W4A16) {
+            float f[8];
+            f[0] = bf16_lo(v[b].x); f[1] = bf16_hi(v[b].x);
+            f[2] = bf16_lo(v[b].y); f[3] = bf16_hi(v[b].y);
+            f[4] = bf16_lo(v[b].z); f[5] = bf16_hi(v[b].z);
+            f[6] = bf16_lo(v[b].w); f[7] = bf16_hi(v[b].w);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) range_bad |= (fabsf(f[e]) > 65504.0f) ? 1u : 0u;
+            hv.x = pack_f16x2(f[0], f[1]);
+            hv.y = pack_f16x2(f[2], f[3]);
+            hv.z = pack_f16x2(f[4], f[5]);
+            hv.w = pack_f16x2(f[6], f[7]);
+          } else {
+            const uint32_t sc = bcast_lo(e4m3x2_to_f16x2(sv[b]));
+            uint32_t q0, q1, q2, q3;
+            e2m1x8_to_f16x2(v[b].x, q0, q1, q2, q3);
+            hv.x = hmul2(q0, sc);
+            hv.y = hmul2(q1, sc);
+            hv.z = hmul2(q2, sc);
+            hv.w = hmul2(q3, sc);
+          }
+        }
+        // columns [k, k + 8): stage c, line lt, MMA pair m of lane (tau % 8, lt)
+        const int c = k / kKS, kk = k % kKS, lt = kk / 256, m = (kk % 256) / 8;
+        act[act_index(c, ng, tau / 8, m, (tau & 7) * 4 + lt)] = hv;
       }
       if (MODE == MOE_W4A16 && range_bad) raise_device_error(MOE_DEVERR_ACT_RANGE);
       named_bar_sync(1, kThreads);
@@ -309,6 +369,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     if (warp >= r.nblk) continue;
+    const float gw = p.w_global ? __ldg(p.w_global + r.e) : 1.0f;  // used by the epilogue
     float acc0[kNG][4], acc1[kNG][4];
 #pragma unroll
     for (int G = 0; G < kNG; ++G)
@@ -337,7 +398,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // ---- block epilogue: scale, round to bf16, transpose, 16-byte stores
     if (!*abort_flag) {
-      const float gw = p.w_global ? p.w_global[r.e] : 1.0f;
       const float f = __fmul_rn(gw, p.g_a);
       uint16_t *st = staging + warp * (kMaxTS * 16);
       auto y = [&](int G, int i) { return __fmul_rn(acc0[G][i] + acc1[G][i], f); };

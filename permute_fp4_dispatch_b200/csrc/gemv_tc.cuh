@@ -131,8 +131,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tbase = *tmem_slot;
 
   const uint32_t U = prefix[A];
-  const uint32_t u_begin = (uint32_t)(((uint64_t)U * blockIdx.x) / gridDim.x);
-  const uint32_t u_end = (uint32_t)(((uint64_t)U * (blockIdx.x + 1)) / gridDim.x);
+  uint32_t u_begin, u_end;
+  cta_round_range(U, RB, kBlocksPerRound, u_begin, u_end);
   const int nchunks = (K + kKC - 1) / kKC;
   const int64_t sf_row_bytes = K / 16;
   const Meta meta{prefix, s_start, s_eid, N};
@@ -144,7 +144,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == kTmaWarp) {
     // ================================================================ TMA producer
-    RoundIter iter{u_begin, u_end, 0, (uint32_t)kTS};
+    RoundIter iter{u_begin, u_end, u_begin < u_end ? expert_of_unit(prefix, A, u_begin) : 0, (uint32_t)kTS};
     Round r;
     uint32_t it = 0;
     const uint64_t policy = l2_evict_first_policy();
@@ -182,7 +182,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kMmaWarp) {
     // ================================================================ MMA issuer
     if (lane == 0) {
-      RoundIter iter{u_begin, u_end, 0, (uint32_t)kTS};
+      RoundIter iter{u_begin, u_end, u_begin < u_end ? expert_of_unit(prefix, A, u_begin) : 0, (uint32_t)kTS};
       Round r;
       uint32_t it = 0, rnd = 0;
       while (iter.next(meta, RB, r)) {
@@ -220,7 +220,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int h = warp >> 2;    // column half of a chunk
     const int row = 32 * q + lane;
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-    RoundIter iter{u_begin, u_end, 0, (uint32_t)kTS};
+    RoundIter iter{u_begin, u_end, u_begin < u_end ? expert_of_unit(prefix, A, u_begin) : 0, (uint32_t)kTS};
     Round r, rn, rp;  // current, next, previous (pending epilogue)
     bool have = iter.next(meta, RB, r);
     bool have_n = have && iter.next(meta, RB, rn);

@@ -424,10 +424,11 @@ moe_status_t moe_grouped_gemv_nvfp4(moe_gemv_mode_t mode, const void *act, const
   // tokens per expert take the tensor-memory variant, whose tcgen05 MMA has a
   // fixed per-instruction cost up to N = 64 and whose passes hold 64 tokens.
   const int ts_mma = maps.sf_tma ? mma::tokens_per_pass(K) : 0;
-  bool use_mma = ts_mma >= 8 && S <= (int64_t)ts_mma * E;
+  const bool mma_ok = ts_mma >= 8 && E <= mma::kMaxActive;
+  bool use_mma = mma_ok && S <= (int64_t)ts_mma * E;
   // test hook: MOE_GEMV_VARIANT=mma|tc forces a variant (both are exact for every input)
   if (const char *v = std::getenv("MOE_GEMV_VARIANT")) {
-    if (v[0] == 'm' && ts_mma >= 8) use_mma = true;
+    if (v[0] == 'm' && mma_ok) use_mma = true;
     if (v[0] == 't') use_mma = false;
   }
   if (use_mma) {
