@@ -67,6 +67,27 @@ def measured_peaks():
     return 6650.0, "profiling-recipe fallback 6.65 TB/s (of fallback)"
 
 
+def profiled_traffic(workload: str):
+    """DRAM bytes per GEMV launch from the committed ncu summary of this
+    workload, or None when there is none or the kernel sources differ from the
+    ones that were profiled (the summary records their sha256)."""
+    import hashlib
+    import re
+    path = os.path.join(ROOT, "profiles", f"grouped_gemv_nvfp4_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m_t = re.search(r"traffic_bytes_per_launch = (\d+)", text)
+    m_h = re.search(r"source_sha256\(([^)]*)\) = ([0-9a-f]{64})", text)
+    if not (m_t and m_h):
+        return None
+    h = hashlib.sha256()
+    for name in m_h.group(1).split("+"):
+        with open(os.path.join(ROOT, "permute_fp4_dispatch_b200", "csrc", name.strip()), "rb") as f:
+            h.update(f.read())
+    return int(m_t.group(1)) if h.hexdigest() == m_h.group(2) else None
+
+
 # ------------------------------------------------------------------ byte model
 def algorithmic_bytes(cfg, mode: str, A: int, R: int, routed_tokens: int) -> dict:
     """Algorithmic HBM bytes per step, per kernel (each input read once, each output
@@ -378,7 +399,8 @@ def run_ours(args, rank, world, local_rank):
                    "l2": "flushed before every step (512 MiB memset outside the timed events)",
                    "graph": "one CUDA graph per step", "parallelism": "replicas"},
         "roofline": {"kernel": "grouped_gemv_nvfp4", "bound": "hbm", "achieved": gemv_gbs,
-                     "peak": peak, "unit": "GB/s", "frac": gemv_gbs / peak, "traffic": None,
+                     "peak": peak, "unit": "GB/s", "frac": gemv_gbs / peak,
+                     "traffic": profiled_traffic(cfg.name),
                      "algorithmic_bytes": bytes_["grouped_gemv"], "us_per_launch": ms_gemv * 1e3,
                      "peak_source": peak_src},
         "pipeline_roofline": {"algorithmic_bytes": total_bytes,

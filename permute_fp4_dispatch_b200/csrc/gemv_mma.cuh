@@ -325,7 +325,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      named_bar_sync(1, kThreads);  // every warp is done with the previous tile
+      if (pass_key != 0xFFFFFFFFu) named_bar_sync(1, kThreads);  // previous tile no longer read
       ng = (r.ntok + 7) / 8;
       if ((int)threadIdx.x < r.ntok) s_pair[threadIdx.x] = my_pair;
       unsigned range_bad = 0;
