@@ -115,21 +115,38 @@ class RoutingPipeline:
         moe_combine(self.expert_out, self.router_weights, self.routing_map, self.N, self.top_k,
                     self.N_out, self.E, self.epi, self.alpha, self.output, stream)
 
-    def run(self, stream=None, gemv_events=None):
-        """All steps in order on one stream.  ``gemv_events`` = (start, end) CUDA
-        events recorded around the GEMV launch, for per-kernel timing."""
-        self.mask(stream)
-        self.create_indices(stream)
-        if self.dispatch:
-            self.dispatch_mxfp4(stream)
+    def run(self, stream=None, gemv_events=None, side_stream=None):
+        """All steps in order.  ``gemv_events`` = (start, end) CUDA events
+        recorded around the GEMV launch, for per-kernel timing.  With
+        ``side_stream``, the MXFP4 dispatch (whose buffer neither the GEMV nor
+        the combine reads) runs there, forked after create_indices and joined
+        at the end; it is enqueued after the GEMV so that the GEMV's
+        persistent CTAs take the SMs first and the dispatch fills the SMs the
+        GEMV frees."""
+        main = stream if stream is not None else torch.cuda.current_stream()
+        self.mask(main)
+        self.create_indices(main)
+        forked = self.dispatch and side_stream is not None
+        if self.dispatch and not forked:
+            self.dispatch_mxfp4(main)
+        if forked:
+            fork = torch.cuda.Event()
+            fork.record(main)
         if self.gemv_mode == MOE_W4A4:
-            self.quantize_activations(stream)
+            self.quantize_activations(main)
         if gemv_events is not None:
-            gemv_events[0].record(stream)
-        self.gemv(stream)
+            gemv_events[0].record(main)
+        self.gemv(main)
         if gemv_events is not None:
-            gemv_events[1].record(stream)
-        self.combine(stream)
+            gemv_events[1].record(main)
+        if forked:
+            side_stream.wait_event(fork)
+            self.dispatch_mxfp4(side_stream)
+            join = torch.cuda.Event()
+            join.record(side_stream)
+        self.combine(main)
+        if forked:
+            main.wait_event(join)
 
     def launches_per_run(self) -> int:
         n = 1 + (1 if self.S <= 16384 else 2) + (1 if self.dispatch else 0)
