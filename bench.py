@@ -283,10 +283,15 @@ def run_ours(args, rank, world, local_rank):
     pipe = RoutingPipeline(cfg.N, cfg.K, cfg.E, cfg.top_k, cfg.N_out, mode=mode,
                            epilogue=cfg.epilogue, device=dev)
     # pinned host copies of the step's inputs (for the end-to-end measurement)
-    h_x = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory()
-    h_ids = torch.from_numpy(ids).pin_memory()
-    h_rw = torch.from_numpy(rw).pin_memory()
-    h_real = torch.tensor([cfg.real], dtype=torch.int32).pin_memory()
+    # a step's inputs live in one pinned host buffer laid out like the device
+    # input arena, so they travel in one copy
+    h_in, h_views = pipe.host_inputs()
+    h_x, h_ids, h_rw, h_real = (h_views[k] for k in ("x", "routing_map", "router_weights",
+                                                       "real_token_count"))
+    h_x.copy_(torch.from_numpy(x.view(np.int16)).view(torch.bfloat16))
+    h_ids.copy_(torch.from_numpy(ids))
+    h_rw.copy_(torch.from_numpy(rw))
+    h_real.fill_(cfg.real)
     h_out = torch.empty((cfg.N, cfg.N_out), dtype=torch.bfloat16).pin_memory()
     pipe.x.copy_(h_x)
     pipe.routing_map.copy_(h_ids)
@@ -359,17 +364,14 @@ def run_ours(args, rank, world, local_rank):
 
     # end to end through the public API, host buffers: H2D inputs, step, D2H output
     e2e_ms = []
-    h2d = h_x.numel() * 2 + h_ids.numel() * 8 + h_rw.numel() * 4 + 4
+    h2d = h_in.numel()   # x, routing map, router weights, real_token_count (+ alignment gaps)
     d2h = h_out.numel() * 2
     for i in range(args.warmup + args.steps):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         with torch.cuda.stream(stream):
             flush.zero_()
             e0.record(stream)
-            pipe.x.copy_(h_x, non_blocking=True)
-            pipe.routing_map.copy_(h_ids, non_blocking=True)
-            pipe.router_weights.copy_(h_rw, non_blocking=True)
-            pipe.real_token_count.copy_(h_real, non_blocking=True)
+            pipe.inputs.copy_(h_in, non_blocking=True)
             graph.replay()
             h_out.copy_(pipe.output, non_blocking=True)
             e1.record(stream)

@@ -5,6 +5,7 @@
  *
  *   moe_mask_padding                 mask CUDA-graph padding rows of the routing map
  *   moe_create_indices               group (token, slot) pairs by expert (CSR)
+ *   moe_mask_and_create_indices      steps 1 and 2 in one call
  *   moe_dispatch_mxfp4               expert-grouped MXFP4 send buffer (1 GPU)
  *   moe_quantize_activations_nvfp4   W4A4 only: bf16 activations -> NVFP4
  *   moe_grouped_gemv_nvfp4           grouped expert GEMV on an NVFP4 library
@@ -119,6 +120,25 @@ MOE_API moe_status_t moe_create_indices(const int64_t *topk_ids, int64_t num_slo
                                 uint32_t *restore_token_order, int32_t *expert_ids,
                                 uint32_t *expert_usage_stats, uint32_t *scales_offset,
                                 void *workspace, size_t ws_bytes, cudaStream_t s);
+
+/* Steps 1 and 2 in one call: exactly moe_mask_padding(routing_map, N,   */
+/* top_k, real_token_count, tp_rank) followed by moe_create_indices on   */
+/* the masked map (num_slots = N * top_k), with the same outputs,        */
+/* including the -1 written into masked rows of routing_map.  When       */
+/* N * top_k <= 1024 both steps run as one single-CTA kernel (one load   */
+/* per slot, no second launch); larger maps take the two-call path.      */
+/* Arguments, limits, workspace and errors: as the two calls (workspace  */
+/* may be NULL when N * top_k <= 1024).                                  */
+MOE_API moe_status_t moe_mask_and_create_indices(int64_t *routing_map, int32_t N, int32_t top_k,
+                                                 const int32_t *real_token_count,
+                                                 int32_t tp_rank, int32_t E,
+                                                 uint32_t *token_expert_order,
+                                                 uint32_t *expert_start_indices,
+                                                 uint32_t *restore_token_order,
+                                                 int32_t *expert_ids,
+                                                 uint32_t *expert_usage_stats,
+                                                 uint32_t *scales_offset, void *workspace,
+                                                 size_t ws_bytes, cudaStream_t s);
 
 /* The same grouping for callers that cannot provide a workspace.  (The   */
 /* method's pages have no counterpart: this is an interface convenience.) */

@@ -23,6 +23,7 @@ __all__ = [
     "MOE_DEVERR_WAIT_TIMEOUT", "MOE_DEVERR_RECV_OVERFLOW", "MOE_DEVERR_ACT_RANGE",
     "moe_mask_padding", "moe_create_indices_workspace_bytes", "moe_create_indices",
     "moe_create_indices_static", "MOE_CREATE_INDICES_STATIC_SCRATCH",
+    "moe_mask_and_create_indices",
     "moe_mxfp4_row_stride", "moe_dispatch_mxfp4", "moe_quantize_activations_nvfp4",
     "moe_quantize_weights_nvfp4", "moe_grouped_gemv_nvfp4", "moe_combine",
     "moe_status_string", "moe_get_device_error", "moe_version",
@@ -52,6 +53,8 @@ _SIGS = {
     "moe_create_indices_workspace_bytes": ([_I64, _I32], _SZ),
     "moe_create_indices": ([_P, _I64, _I32, _P, _P, _P, _P, _P, _P, _P, _SZ, _P], _I32),
     "moe_create_indices_static": ([_P, _I64, _I32, _P, _P, _P, _P, _P, _P, _P], _I32),
+    "moe_mask_and_create_indices": ([_P, _I32, _I32, _P, _I32, _I32, _P, _P, _P, _P, _P, _P,
+                                     _P, _SZ, _P], _I32),
     "moe_mxfp4_row_stride": ([_I32], _SZ),
     "moe_dispatch_mxfp4": ([_P, _I32, _I32, _I32, _I32, _P, _P, _P, _P, _P, _I64, _P, _P], _I32),
     "moe_quantize_activations_nvfp4": ([_P, _I32, _I32, _F32, _P, _P, _P], _I32),
@@ -132,6 +135,19 @@ def moe_create_indices(topk_ids, num_slots: int, E: int, token_expert_order,
         _ptr(topk_ids), num_slots, E, _ptr(token_expert_order), _ptr(expert_start_indices),
         _ptr(restore_token_order), _ptr(expert_ids), _ptr(expert_usage_stats),
         _ptr(scales_offset), _ptr(workspace), ws_bytes, _stream(stream)), "moe_create_indices")
+
+
+def moe_mask_and_create_indices(routing_map, N: int, top_k: int, real_token_count,
+                                tp_rank: int, E: int, token_expert_order, expert_start_indices,
+                                restore_token_order, expert_ids, expert_usage_stats,
+                                scales_offset, workspace, ws_bytes: int, stream=None):
+    """moe_mask_padding followed by moe_create_indices on the masked map, one
+    kernel when N * top_k <= 1024."""
+    _check(library().moe_mask_and_create_indices(
+        _ptr(routing_map), N, top_k, _ptr(real_token_count), tp_rank, E,
+        _ptr(token_expert_order), _ptr(expert_start_indices), _ptr(restore_token_order),
+        _ptr(expert_ids), _ptr(expert_usage_stats), _ptr(scales_offset), _ptr(workspace),
+        ws_bytes, _stream(stream)), "moe_mask_and_create_indices")
 
 
 MOE_CREATE_INDICES_STATIC_SCRATCH = 262144

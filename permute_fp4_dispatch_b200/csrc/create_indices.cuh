@@ -263,5 +263,142 @@ __global__ void __launch_bounds__(kThreads, 1)
   warp_scatter(ids, lo, hi, E, s, my_hist, order, restore);
 }
 
+// ---------------------------------------------------------------- steps 1 + 2 fused
+// Up to kTinySlots slots: one CTA of kThreads threads, one slot per thread.
+// Thread p applies the step-1 mask to its slot (rows with
+// row + tp_rank * N >= *real_token_count are written back as -1), keeps the
+// resulting id in a register from its single load to the scatter, and the
+// grouping then follows the same counting sort as above with the cross-warp
+// prefix done by warp shuffles (experts striped over warps, one lane per
+// source warp) and the CSR compaction done in one combined block scan.
+constexpr int kTinySlots = kThreads;
+
+__host__ __device__ inline int tiny_hist_stride(int E) { return ((E + 1) / 2 | 1) * 2; }
+
+__host__ __device__ inline size_t tiny_smem_bytes(int E) {
+  return ((size_t)kWarps * tiny_hist_stride(E) * 2 + 15) / 16 * 16 + (size_t)E * 8;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    mask_create_indices_tiny_kernel(int64_t *__restrict__ ids, int32_t N, int32_t top_k,
+                                    const int32_t *__restrict__ real_count, int32_t tp_rank,
+                                    int E, uint32_t *__restrict__ order,
+                                    uint32_t *__restrict__ start, uint32_t *__restrict__ restore,
+                                    int32_t *__restrict__ expert_ids,
+                                    uint32_t *__restrict__ stats,
+                                    uint32_t *__restrict__ scales_offset) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  const int WS = tiny_hist_stride(E);
+  uint16_t *whist = reinterpret_cast<uint16_t *>(smem_raw);
+  uint32_t *cnt = reinterpret_cast<uint32_t *>(smem_raw +
+                                               ((size_t)kWarps * WS * 2 + 15) / 16 * 16);
+  uint32_t *off = cnt + E;
+  __shared__ uint32_t wsum[4][kWarps];
+  __shared__ uint32_t totals[4];
+  const int p = threadIdx.x, warp = p >> 5, lane = p & 31;
+  const int S = N * top_k;
+  const unsigned lt = (1u << lane) - 1u;
+
+  // step 1 + key: one load per slot
+  int key = -1;
+  if (p < S) {
+    const int row = p / top_k;
+    if ((int64_t)row + (int64_t)tp_rank * N >= (int64_t)*real_count) {
+      ids[p] = -1;
+    } else {
+      const int64_t id = ids[p];
+      key = (id >= 0 && id < E) ? (int)id : -1;
+    }
+  }
+  for (int i = p; i < kWarps * WS; i += kThreads) whist[i] = 0;
+  __syncthreads();
+  const unsigned peers = __match_any_sync(0xffffffffu, key);
+  if (key >= 0 && lane == __ffs(peers) - 1) whist[warp * WS + key] = (uint16_t)__popc(peers);
+  __syncthreads();
+  // per expert: exclusive prefix over the 32 warps (lane = source warp)
+  for (int e = warp; e < E; e += kWarps) {
+    const uint32_t c = whist[lane * WS + e];
+    uint32_t x = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    whist[lane * WS + e] = (uint16_t)(x - c);
+    if (lane == 31) cnt[e] = x;
+  }
+  __syncthreads();
+  // CSR over experts: one block scan of (active flag, count, count padded to 128) and a max
+  const uint32_t c = p < E ? cnt[p] : 0u;
+  uint32_t v0 = c > 0 ? 1u : 0u, v1 = c, v2 = (c + 127u) / 128u * 128u, mx = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y0 = __shfl_up_sync(0xffffffffu, v0, o);
+    const uint32_t y1 = __shfl_up_sync(0xffffffffu, v1, o);
+    const uint32_t y2 = __shfl_up_sync(0xffffffffu, v2, o);
+    if (lane >= o) { v0 += y0; v1 += y1; v2 += y2; }
+    mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+  if (lane == 31) {
+    wsum[0][warp] = v0;
+    wsum[1][warp] = v1;
+    wsum[2][warp] = v2;
+    wsum[3][warp] = mx;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    uint32_t a = wsum[0][lane], r = wsum[1][lane], q = wsum[2][lane], m = wsum[3][lane];
+    const uint32_t a0 = a, r0 = r, q0 = q;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t ya = __shfl_up_sync(0xffffffffu, a, o);
+      const uint32_t yr = __shfl_up_sync(0xffffffffu, r, o);
+      const uint32_t yq = __shfl_up_sync(0xffffffffu, q, o);
+      if (lane >= o) { a += ya; r += yr; q += yq; }
+      m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+    }
+    wsum[0][lane] = a - a0;
+    wsum[1][lane] = r - r0;
+    wsum[2][lane] = q - q0;
+    if (lane == 31) {
+      totals[0] = a;
+      totals[1] = r;
+      totals[2] = q;
+      totals[3] = m;
+    }
+  }
+  __syncthreads();
+  const uint32_t A = totals[0], R = totals[1], P = totals[2];
+  if (p < E) {
+    const uint32_t pos = wsum[0][warp] + v0 - (c > 0 ? 1u : 0u);
+    const uint32_t o = wsum[1][warp] + v1 - c;
+    off[p] = o;
+    if (c > 0) {
+      expert_ids[pos] = p;
+      start[pos] = o;
+      if (scales_offset) scales_offset[pos] = wsum[2][warp] + v2 - (c + 127u) / 128u * 128u;
+    }
+  }
+  for (int i = (int)A + p; i <= E; i += kThreads) {  // entries [A, E] (E may equal kThreads)
+    if (i < E) expert_ids[i] = -1;
+    start[i] = R;
+    if (scales_offset) scales_offset[i] = P;
+  }
+  if (p == 0) {
+    stats[0] = totals[3];
+    stats[1] = A;
+  }
+  __syncthreads();
+  // stable scatter
+  if (key >= 0) {
+    const uint32_t dest = off[key] + whist[warp * WS + key] + __popc(peers & lt);
+    order[dest] = (uint32_t)p;
+    restore[p] = dest;
+  } else if (p < S) {
+    restore[p] = 0xFFFFFFFFu;
+  }
+  if (p >= (int)R && p < S) order[p] = 0xFFFFFFFFu;
+}
+
 }  // namespace idx
 }  // namespace moe

@@ -278,6 +278,42 @@ moe_status_t moe_create_indices(const int64_t *topk_ids, int64_t num_slots, int3
   return launch_status();
 }
 
+moe_status_t moe_mask_and_create_indices(int64_t *routing_map, int32_t N, int32_t top_k,
+                                         const int32_t *real_token_count, int32_t tp_rank,
+                                         int32_t E, uint32_t *token_expert_order,
+                                         uint32_t *expert_start_indices,
+                                         uint32_t *restore_token_order, int32_t *expert_ids,
+                                         uint32_t *expert_usage_stats, uint32_t *scales_offset,
+                                         void *workspace, size_t ws_bytes, cudaStream_t s) {
+  using namespace moe::idx;
+  if (N < 0 || top_k < 1 || tp_rank < 0 || !real_token_count) return MOE_ERR_INVALID_ARG;
+  const int64_t S = (int64_t)N * top_k;
+  if (S > kTinySlots) {
+    moe_status_t st = moe_mask_padding(routing_map, N, top_k, real_token_count, tp_rank, s);
+    if (st != MOE_OK) return st;
+    return moe_create_indices(routing_map, S, E, token_expert_order, expert_start_indices,
+                              restore_token_order, expert_ids, expert_usage_stats, scales_offset,
+                              workspace, ws_bytes, s);
+  }
+  if (E < 1 || E > 1024) return MOE_ERR_INVALID_ARG;
+  if (!expert_start_indices || !expert_ids || !expert_usage_stats) return MOE_ERR_INVALID_ARG;
+  if (S > 0 && (!routing_map || !token_expert_order || !restore_token_order))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned(routing_map, 8) || !aligned(real_token_count, 4) ||
+      !aligned(token_expert_order, 4) || !aligned(restore_token_order, 4) ||
+      !aligned(expert_start_indices, 4) || !aligned(expert_ids, 4) ||
+      !aligned(expert_usage_stats, 4) || !aligned(scales_offset, 4))
+    return MOE_ERR_INVALID_ARG;
+  moe_status_t st = check_device();
+  if (st != MOE_OK) return st;
+  const size_t smem = tiny_smem_bytes(E);
+  if ((st = set_smem(mask_create_indices_tiny_kernel, smem)) != MOE_OK) return st;
+  mask_create_indices_tiny_kernel<<<1, kThreads, smem, s>>>(
+      routing_map, N, top_k, real_token_count, tp_rank, E, token_expert_order,
+      expert_start_indices, restore_token_order, expert_ids, expert_usage_stats, scales_offset);
+  return launch_status();
+}
+
 // ------------------------------------------------------------------ step 3
 size_t moe_mxfp4_row_stride(int32_t K) {
   if (K <= 0) return 0;

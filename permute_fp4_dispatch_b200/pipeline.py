@@ -5,7 +5,7 @@ the library's kernels do all the work.
     pipe.quantize_weights(w_f32_expert_slices)      # offline, once
     pipe.x.copy_(...); pipe.routing_map.copy_(...); pipe.router_weights.copy_(...)
     pipe.real_token_count.fill_(real)
-    pipe.run()                                      # mask -> indices -> dispatch -> GEMV -> combine
+    pipe.run()                                      # mask + indices -> dispatch || GEMV -> combine
     pipe.output                                     # bf16 [N, N_out]
 
 Every buffer is allocated once at construction, so ``run`` allocates
@@ -17,10 +17,30 @@ import torch
 
 from . import (MOE_EPI_IDENTITY, MOE_EPI_NONE, MOE_EPI_SCALE, MOE_W4A4, MOE_W4A16,
                moe_combine, moe_create_indices, moe_create_indices_workspace_bytes,
+               moe_mask_and_create_indices,
                moe_dispatch_mxfp4, moe_grouped_gemv_nvfp4, moe_mask_padding,
                moe_mxfp4_row_stride, moe_quantize_activations_nvfp4, moe_quantize_weights_nvfp4)
 
 EPILOGUES = {"none": MOE_EPI_NONE, "identity": MOE_EPI_IDENTITY, "scale": MOE_EPI_SCALE}
+
+
+def _arena_layout(fields, align: int = 256):
+    """Byte offsets of the fields (name, shape, dtype), each aligned to
+    ``align``; returns (entries, total bytes)."""
+    entries, off = [], 0
+    for name, shape, dtype in fields:
+        n = 1
+        for d in shape:
+            n *= d
+        nbytes = n * torch.empty((), dtype=dtype).element_size()
+        entries.append((name, shape, dtype, off, nbytes))
+        off += (nbytes + align - 1) // align * align
+    return entries, max(off, align)
+
+
+def _arena_views(buf: torch.Tensor, entries):
+    return {name: buf[off:off + nbytes].view(dtype).view(shape)
+            for name, shape, dtype, off, nbytes in entries}
 
 
 class RoutingPipeline:
@@ -41,11 +61,14 @@ class RoutingPipeline:
         S = N * top_k
         self.S = S
         u8, i32, i64 = torch.uint8, torch.int32, torch.int64
-        # inputs
-        self.x = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
-        self.routing_map = torch.empty((N, top_k), dtype=i64, device=dev)
-        self.router_weights = torch.empty((N, top_k), dtype=torch.float32, device=dev)
-        self.real_token_count = torch.zeros(1, dtype=i32, device=dev)
+        # inputs: views into one byte arena, so a step's inputs travel from a
+        # pinned host mirror (host_inputs()) in a single copy
+        self._input_layout = _arena_layout([
+            ("x", (N, K), torch.bfloat16), ("routing_map", (N, top_k), i64),
+            ("router_weights", (N, top_k), torch.float32), ("real_token_count", (1,), i32)])
+        self.inputs = torch.zeros(self._input_layout[1], dtype=u8, device=dev)
+        for name, t in _arena_views(self.inputs, self._input_layout[0]).items():
+            setattr(self, name, t)
         # expert library
         self.wq = torch.empty((E, N_out, K // 2), dtype=u8, device=dev)
         self.sfw = torch.empty((E, N_out, K // 16), dtype=u8, device=dev)
@@ -74,6 +97,14 @@ class RoutingPipeline:
         # step 5
         self.output = torch.empty((N, N_out), dtype=torch.bfloat16, device=dev)
 
+    def host_inputs(self):
+        """A pinned host byte buffer laid out like ``inputs`` and its typed
+        views (x, routing_map, router_weights, real_token_count):
+        ``pipe.inputs.copy_(buf, non_blocking=True)`` moves a whole step's
+        inputs in one transfer."""
+        buf = torch.zeros(self._input_layout[1], dtype=torch.uint8, pin_memory=True)
+        return buf, _arena_views(buf, self._input_layout[0])
+
     # ------------------------------------------------------------ weights
     def quantize_weights(self, w_f32: torch.Tensor, expert_base: int = 0, stream=None):
         """Quantise fp32 weights [e, N_out, K] (device) into experts [base, base + e)."""
@@ -94,6 +125,13 @@ class RoutingPipeline:
                            self.expert_start_indices, self.restore_token_order, self.expert_ids,
                            self.expert_usage_stats, self.scales_offset, self.workspace,
                            self.ws_bytes, stream)
+
+    def mask_and_create_indices(self, stream=None):
+        moe_mask_and_create_indices(self.routing_map, self.N, self.top_k, self.real_token_count,
+                                    self.tp_rank, self.E, self.token_expert_order,
+                                    self.expert_start_indices, self.restore_token_order,
+                                    self.expert_ids, self.expert_usage_stats, self.scales_offset,
+                                    self.workspace, self.ws_bytes, stream)
 
     def dispatch_mxfp4(self, stream=None):
         moe_dispatch_mxfp4(self.x, self.N, self.K, self.top_k, self.E, self.restore_token_order,
@@ -124,8 +162,7 @@ class RoutingPipeline:
         persistent CTAs take the SMs first and the dispatch fills the SMs the
         GEMV frees."""
         main = stream if stream is not None else torch.cuda.current_stream()
-        self.mask(main)
-        self.create_indices(main)
+        self.mask_and_create_indices(main)
         forked = self.dispatch and side_stream is not None
         if self.dispatch and not forked:
             self.dispatch_mxfp4(main)
@@ -149,6 +186,8 @@ class RoutingPipeline:
             main.wait_event(join)
 
     def launches_per_run(self) -> int:
-        n = 1 + (1 if self.S <= 16384 else 2) + (1 if self.dispatch else 0)
+        # mask + create_indices: one fused kernel up to 1024 slots, else mask and 1-2 kernels
+        front = 1 if self.S <= 1024 else 1 + (1 if self.S <= 16384 else 2)
+        n = front + (1 if self.dispatch else 0)
         n += 1 if self.gemv_mode == MOE_W4A4 else 0
         return n + 2

@@ -78,6 +78,53 @@ def test_create_indices_deterministic_and_skewed():
         check_indices(gpu_create_indices(ids, 64), ref, ids.size)
 
 
+# ------------------------------------------------------------------ steps 1 + 2 fused
+def gpu_mask_and_create_indices(m: np.ndarray, E: int, real: int, tp: int):
+    N, k = m.shape
+    S = N * k
+    t = dev(m.astype(np.int64)) if S else torch.empty(1, dtype=torch.int64, device="cuda")
+    cnt = torch.tensor([real], dtype=torch.int32, device="cuda")
+    order = torch.full((max(S, 1),), 0x5A5A5A5A, dtype=torch.int32, device="cuda")
+    restore = torch.full((max(S, 1),), 0x5A5A5A5A, dtype=torch.int32, device="cuda")
+    start = torch.full((E + 1,), 0x5A5A5A5A, dtype=torch.int32, device="cuda")
+    eids = torch.full((E,), 0x5A5A5A5A, dtype=torch.int32, device="cuda")
+    stats = torch.full((2,), 0x5A5A5A5A, dtype=torch.int32, device="cuda")
+    soff = torch.full((E + 1,), 0x5A5A5A5A, dtype=torch.int32, device="cuda")
+    ws_bytes = moe.moe_create_indices_workspace_bytes(S, E)
+    ws = torch.full((max(ws_bytes, 256),), 0x5A, dtype=torch.uint8, device="cuda")
+    moe.moe_mask_and_create_indices(t, N, k, cnt, tp, E, order, start, restore, eids, stats,
+                                    soff, ws, ws_bytes)
+    out = dict(token_expert_order=host_u32(order)[:S], expert_start_indices=host_u32(start),
+               restore_token_order=host_u32(restore)[:S], expert_ids=eids.cpu().numpy(),
+               expert_usage_stats=host_u32(stats), scales_offset=host_u32(soff))
+    return t.cpu().numpy()[:S].reshape(N, k) if S else m, out
+
+
+@pytest.mark.parametrize("N,k,E,real,tp", [
+    (128, 8, 128, 128, 0),      # decode-sized, nothing masked
+    (128, 8, 128, 77, 0),       # ragged real count
+    (13, 2, 8, 9, 1),           # tp_rank offset: rows 0.. of rank 1 start at 13
+    (64, 16, 1024, 50, 0),      # E = 1024 (one expert per thread)
+    (1024, 1, 3, 1000, 0),      # top_k = 1, S = 1024 exactly
+    (37, 3, 12, -5, 0),         # real <= 0: everything masked
+    (37, 3, 12, 4000, 0),       # real > N: nothing masked
+    (1, 1, 1, 1, 0),            # minimal
+    (129, 8, 64, 100, 0),       # S = 1032 > 1024: the two-call path
+])
+def test_mask_and_create_indices_equals_two_steps(N, k, E, real, tp):
+    rng = np.random.default_rng(N * 31 + k + E)
+    m = rng.integers(-2, E + 2, (N, k)).astype(np.int64)   # includes -1 and out-of-range ids
+    masked_ref = oracle.mask_padding(m, real, tp)
+    ref = oracle.create_indices(masked_ref.reshape(-1), E)
+    masked_gpu, got = gpu_mask_and_create_indices(m, E, real, tp)
+    np.testing.assert_array_equal(masked_gpu, masked_ref)
+    check_indices(got, ref, N * k)
+    # and byte for byte what the separate entry points give
+    sep = gpu_create_indices(masked_ref, E)
+    for key in sep:
+        np.testing.assert_array_equal(got[key], sep[key], err_msg=key)
+
+
 # ------------------------------------------------------------------ codecs (exhaustive)
 def all_finite_bf16(shuffle_seed=None) -> np.ndarray:
     bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
