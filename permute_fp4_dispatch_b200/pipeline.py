@@ -63,9 +63,11 @@ class RoutingPipeline:
         u8, i32, i64 = torch.uint8, torch.int32, torch.int64
         # inputs: views into one byte arena, so a step's inputs travel from a
         # pinned host mirror (host_inputs()) in a single copy
+        # (the routing inputs come first: they can be copied ahead of x)
         self._input_layout = _arena_layout([
-            ("x", (N, K), torch.bfloat16), ("routing_map", (N, top_k), i64),
-            ("router_weights", (N, top_k), torch.float32), ("real_token_count", (1,), i32)])
+            ("routing_map", (N, top_k), i64), ("router_weights", (N, top_k), torch.float32),
+            ("real_token_count", (1,), i32), ("x", (N, K), torch.bfloat16)])
+        self.routing_bytes = self._input_layout[0][3][3]   # offset of x in the arena
         self.inputs = torch.zeros(self._input_layout[1], dtype=u8, device=dev)
         for name, t in _arena_views(self.inputs, self._input_layout[0]).items():
             setattr(self, name, t)
@@ -153,16 +155,20 @@ class RoutingPipeline:
         moe_combine(self.expert_out, self.router_weights, self.routing_map, self.N, self.top_k,
                     self.N_out, self.E, self.epi, self.alpha, self.output, stream)
 
-    def run(self, stream=None, gemv_events=None, side_stream=None):
+    def run(self, stream=None, gemv_events=None, side_stream=None, x_ready=None):
         """All steps in order.  ``gemv_events`` = (start, end) CUDA events
         recorded around the GEMV launch, for per-kernel timing.  With
         ``side_stream``, the MXFP4 dispatch (whose buffer neither the GEMV nor
         the combine reads) runs there, forked after create_indices and joined
         at the end; it is enqueued after the GEMV so that the GEMV's
         persistent CTAs take the SMs first and the dispatch fills the SMs the
-        GEMV frees."""
+        GEMV frees.  ``x_ready`` (a CUDA event) holds back the steps that read
+        the activations -- dispatch, activation quantisation, GEMV -- until x
+        has arrived; mask and create_indices run before it."""
         main = stream if stream is not None else torch.cuda.current_stream()
         self.mask_and_create_indices(main)
+        if x_ready is not None:
+            main.wait_event(x_ready)
         forked = self.dispatch and side_stream is not None
         if self.dispatch and not forked:
             self.dispatch_mxfp4(main)
