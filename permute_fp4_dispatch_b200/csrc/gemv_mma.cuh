@@ -282,7 +282,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     ++produced;
     if (++pc == nst) next_own_round();
   };
-  for (int s = 0; s < kSlots; ++s) produce();
+  // the first stages are requested right after the first pass's activation
+  // loads, so the small gathers are not queued behind the weight stream
+  bool primed = false;
 
   // ---- consumer side
   const int g = lane >> 2, t = lane & 3;
@@ -324,6 +326,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
+      }
+      if (!primed) {
+        for (int st = 0; st < kSlots; ++st) produce();
+        primed = true;
       }
       if (pass_key != 0xFFFFFFFFu) named_bar_sync(1, kThreads);  // previous tile no longer read
       ng = (r.ntok + 7) / 8;

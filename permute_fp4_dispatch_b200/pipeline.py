@@ -159,12 +159,11 @@ class RoutingPipeline:
         """All steps in order.  ``gemv_events`` = (start, end) CUDA events
         recorded around the GEMV launch, for per-kernel timing.  With
         ``side_stream``, the MXFP4 dispatch (whose buffer neither the GEMV nor
-        the combine reads) runs there, forked after create_indices and joined
-        at the end; it is enqueued after the GEMV so that the GEMV's
-        persistent CTAs take the SMs first and the dispatch fills the SMs the
-        GEMV frees.  ``x_ready`` (a CUDA event) holds back the steps that read
-        the activations -- dispatch, activation quantisation, GEMV -- until x
-        has arrived; mask and create_indices run before it."""
+        the combine reads) runs there, forked after the GEMV and joined at the
+        end, so it overlaps the combine instead of holding SMs the GEMV's
+        persistent CTAs need.  ``x_ready`` (a CUDA event) holds back the steps
+        that read the activations -- dispatch, activation quantisation, GEMV --
+        until x has arrived; mask and create_indices run before it."""
         main = stream if stream is not None else torch.cuda.current_stream()
         self.mask_and_create_indices(main)
         if x_ready is not None:
@@ -172,9 +171,6 @@ class RoutingPipeline:
         forked = self.dispatch and side_stream is not None
         if self.dispatch and not forked:
             self.dispatch_mxfp4(main)
-        if forked:
-            fork = torch.cuda.Event()
-            fork.record(main)
         if self.gemv_mode == MOE_W4A4:
             self.quantize_activations(main)
         if gemv_events is not None:
@@ -183,6 +179,8 @@ class RoutingPipeline:
         if gemv_events is not None:
             gemv_events[1].record(main)
         if forked:
+            fork = torch.cuda.Event()
+            fork.record(main)
             side_stream.wait_event(fork)
             self.dispatch_mxfp4(side_stream)
             join = torch.cuda.Event()
