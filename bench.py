@@ -426,7 +426,7 @@ def run_ours(args, rank, world, local_rank):
                    "E": cfg.E, "top_k": cfg.top_k, "N_out": cfg.N_out, "mode": mode,
                    "routed_pairs": R, "active_experts": A,
                    "l2": "flushed before every step (512 MiB memset outside the timed events)",
-                   "graph": "one CUDA graph per step (dispatch on a forked stream, concurrent with the GEMV)",
+                   "graph": "one CUDA graph per step (dispatch on a forked stream after the GEMV, beside the combine)",
                    "parallelism": "replicas"},
         "roofline": {"kernel": "grouped_gemv_nvfp4", "bound": "hbm", "achieved": gemv_gbs,
                      "peak": peak, "unit": "GB/s", "frac": gemv_gbs / peak,
