@@ -58,6 +58,23 @@ def parse_args():
     return ap.parse_args()
 
 
+def max_over_ranks(value: float, world: int, device="cpu") -> float:
+    """The largest value over the ranks (a replica job's time is its slowest
+    replica's); with one rank, the value itself."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(units_per_rank: int, world: int, ms: float) -> float:
+    """Whole-job throughput: every rank processes units_per_rank in ms."""
+    return world * units_per_rank / (ms * 1e-3)
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -355,12 +372,8 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize()
     barrier()
     clocks = clk.summary()
-    ms_step = float(np.mean(t_step))
+    ms_step = max_over_ranks(float(np.mean(t_step)), world, dev)
     ms_gemv = float(np.mean(t_gemv))
-    if world > 1:
-        t = torch.tensor([ms_step], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step = float(t.item())
 
     # end to end through the public API, host buffers: one CUDA graph per step
     # holding the H2D copies of the step's inputs from pinned memory (routing
@@ -404,11 +417,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     # the host copy of the last step's output is the device result
     assert torch.equal(h_out.view(torch.int16), pipe.output.cpu().view(torch.int16))
-    e2e_step = float(np.mean(e2e_ms))
-    if world > 1:
-        t = torch.tensor([e2e_step], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_step = float(t.item())
+    e2e_step = max_over_ranks(float(np.mean(e2e_ms)), world, dev)
 
     peak, peak_src = measured_peaks()
     bytes_ = algorithmic_bytes(cfg, mode, A, R, routed_tokens)
@@ -416,7 +425,7 @@ def run_ours(args, rank, world, local_rank):
     total_bytes = sum(bytes_.values())
     line = {
         "metric": "routed token-expert pairs/s end-to-end at 1 B200",
-        "value": world * R / (ms_step * 1e-3),
+        "value": job_rate(R, world, ms_step),
         "unit": "routed pairs/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -437,7 +446,7 @@ def run_ours(args, rank, world, local_rank):
                               "achieved_gbs": total_bytes / (ms_step * 1e-3) / 1e9,
                               "frac": total_bytes / (ms_step * 1e-3) / 1e9 / peak,
                               "bytes_by_kernel": bytes_},
-        "e2e": {"value": world * R / (e2e_step * 1e-3), "unit": "routed pairs/s",
+        "e2e": {"value": job_rate(R, world, e2e_step), "unit": "routed pairs/s",
                 "ms_per_step": e2e_step, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": pipe.launches_per_run() * args.steps,
         "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
