@@ -16,9 +16,9 @@
 //     hide each other's load and dependency latencies.  A stage is 16 rows x
 //     1024 codes:
 //     one 4-D TMA box (16 rows x 4 lines of 128 bytes, 512 contiguous bytes
-//     per row, 128-byte swizzle, L2 evict-first) issued by lane 0, plus the
-//     stage's 16 x 64 E4M3 scale bytes by per-lane 16-byte cp.async, both
-//     completing on the stage's mbarrier.  The TMA engine's cost grows with
+//     per row, 128-byte swizzle, L2 evict-first) plus one 3-D box of the
+//     stage's 16 x 64 E4M3 scale bytes, both issued by lane 0 and completing
+//     on the stage's mbarrier.  The TMA engine's cost grows with
 //     the number of contiguous runs it fetches; 512-byte runs stream at the
 //     rate of plain bulk copies where 128-byte runs do not.
 //   * Lane (g, t) owns line t of rows g and g + 8.  A line index in the box is
@@ -194,7 +194,8 @@ struct RoundWalk {
 
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
-    grouped_gemv_mma_kernel(const Params p, const int ts, const __grid_constant__ CUtensorMap tmap_w) {
+    grouped_gemv_mma_kernel(const Params p, const int ts, const __grid_constant__ CUtensorMap tmap_w,
+                            const __grid_constant__ CUtensorMap tmap_sf) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -206,6 +207,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t *s_pair = reinterpret_cast<uint32_t *>(smem + kOffPair);
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + kOffBar);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffMisc);
+  uint32_t *s_range = reinterpret_cast<uint32_t *>(smem + kOffMisc + 4);
 
   const int warp = threadIdx.x >> 5;
   const int lane = (int)lane_id();
@@ -220,27 +222,37 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (i < A) s_eid[i] = p.eids[i];
   }
   __syncthreads();
-  if (warp == 0) build_prefix(prefix, s_start, A, (uint32_t)ts, RB, lane);
+  if (warp == 0) {
+    build_prefix(prefix, s_start, A, (uint32_t)ts, RB, lane);
+    __syncwarp();
+    if (lane == 0) {  // the CTA's share of the units, computed once
+      uint32_t u0, u1;
+      cta_pass_range(prefix[A], RB, kCW, u0, u1);
+      s_range[0] = u0;
+      s_range[1] = u1;
+    }
+  }
   if (threadIdx.x == 0) {
-    // one arrival with the TMA byte count + one cp.async arrival per lane
-    for (int i = 0; i < kCW * kSlots; ++i) mbar_init(&full[i], 33u);
+    // one arrival with the byte count of the stage's two TMA boxes
+    for (int i = 0; i < kCW * kSlots; ++i) mbar_init(&full[i], 1u);
     *abort_flag = 0;
     fence_mbar_init();
   }
   __syncthreads();
 
-  uint32_t u_begin, u_end;
-  cta_pass_range(prefix[A], RB, kCW, u_begin, u_end);
+  const uint32_t u_begin = s_range[0], u_end = s_range[1];
   if (u_begin >= u_end) return;
   const int nst = (K + kKS - 1) / kKS;  // stages per block
   const int lines_total = K / 256;
-  const int64_t sf_row_bytes = K / 16;
   const Meta meta{prefix, s_start, s_eid, N};
   uint8_t *wring = smem + kOffW + (size_t)warp * kSlots * kStageW;
   uint8_t *sring = smem + kOffSF + (size_t)warp * kSlots * kStageSF;
   uint64_t *wfull = full + warp * kSlots;
   const uint64_t policy = l2_evict_first_policy();
-  if (lane == 0) prefetch_tmap(&tmap_w);
+  if (lane == 0) {
+    prefetch_tmap(&tmap_w);
+    prefetch_tmap(&tmap_sf);
+  }
 
   // ---- producer side of this warp's pipeline: the next (round, stage) of its blocks
   RoundWalk piter;
@@ -268,17 +280,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *bar = &wfull[slot];
     const int n0 = pr.n0 + 16 * warp;
     if (lane == 0) {
-      mbar_arrive_expect_tx(bar, (uint32_t)kStageW);
+      mbar_arrive_expect_tx(bar, (uint32_t)(kStageW + kStageSF));
       tma_load_4d(sw, &tmap_w, 0, pc * kLines, n0, pr.e, bar, policy);
+      // scales: 16 rows x 4 words (one 16-byte group per line), rows beyond N and
+      // lines beyond K read as zero
+      tma_load_3d(ssf, &tmap_sf, pc * kLines * 4, n0, pr.e, bar, policy);
     }
-    for (int piece = lane; piece < 16 * kLines; piece += 32) {
-      const int r = piece / kLines, j = piece % kLines;
-      const int line = pc * kLines + j;
-      if (n0 + r < N && line < lines_total)
-        cp_async16(ssf + r * kRowSF + j * 16,
-                   p.sfw + ((int64_t)pr.e * N + n0 + r) * sf_row_bytes + line * 16);
-    }
-    cp_async_mbar_arrive_noinc(bar);
     ++produced;
     if (++pc == nst) next_own_round();
   };

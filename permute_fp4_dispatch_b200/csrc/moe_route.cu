@@ -133,6 +133,21 @@ bool encode_lines_4d(CUtensorMap *m, const void *base, uint64_t K, uint64_t N, u
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D uint32 map over the scales [E][N][K/16 bytes] seen as [E][N][K/64 words];
+// box = 16 rows x `words` words, no swizzle.  Needs K % 256 == 0 (16-byte rows).
+bool encode_scale_words_3d(CUtensorMap *m, const void *base, uint64_t K, uint64_t N, uint64_t E,
+                           uint32_t words) {
+  auto fn = tensor_map_encoder();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {K / 64, N, E};
+  const cuuint64_t strides[2] = {K / 16, (K / 16) * N};
+  const cuuint32_t box[3] = {words, 16, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<void *>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Descriptors of the expert library, cached by (pointers, shape): encoding
 // costs a driver call, and graph replays reuse the captured parameters anyway.
 struct LibMaps {
@@ -140,7 +155,7 @@ struct LibMaps {
   int E = 0, N = 0, K = 0;
   bool sf_tma = false;  // K % 256 == 0: scale boxes for the tensor-memory variant,
                         // and the line map of the decode variant
-  CUtensorMap tw, tsf, tlines;
+  CUtensorMap tw, tsf, tlines, tsf_lines;
 };
 constexpr int kMapCache = 8;
 LibMaps g_maps[kMapCache];
@@ -163,6 +178,7 @@ bool library_maps(const uint8_t *w, const uint8_t *sfw, int E, int N, int K, Lib
   m.sf_tma = (K % 256) == 0;
   std::memset(&m.tsf, 0, sizeof m.tsf);
   std::memset(&m.tlines, 0, sizeof m.tlines);
+  std::memset(&m.tsf_lines, 0, sizeof m.tsf_lines);
   // the tensor-memory variant reads 16-row x 128-byte weight boxes and 16-row x 16-byte scale boxes
   static_assert(moe::gemv::tc::kWStride == 128 && moe::gemv::tc::kSFStride == 16, "box width");
   if (!encode_u8_3d(&m.tw, w, (uint64_t)K / 2, (uint64_t)N, (uint64_t)E, 128, 16,
@@ -173,6 +189,9 @@ bool library_maps(const uint8_t *w, const uint8_t *sfw, int E, int N, int K, Lib
     return false;
   if (m.sf_tma && !encode_lines_4d(&m.tlines, w, (uint64_t)K, (uint64_t)N, (uint64_t)E,
                                    (uint32_t)moe::gemv::mma::kLines))
+    return false;
+  if (m.sf_tma && !encode_scale_words_3d(&m.tsf_lines, sfw, (uint64_t)K, (uint64_t)N, (uint64_t)E,
+                                         (uint32_t)moe::gemv::mma::kLines * 4))
     return false;
   g_maps[g_maps_next] = m;
   g_maps_next = (g_maps_next + 1) % kMapCache;
@@ -468,11 +487,12 @@ moe_status_t moe_grouped_gemv_nvfp4(moe_gemv_mode_t mode, const void *act, const
     if (v[0] == 't') use_mma = false;
   }
   if (use_mma) {
-    void (*kern)(const Params, const int, const CUtensorMap) =
+    void (*kern)(const Params, const int, const CUtensorMap, const CUtensorMap) =
         mode == MOE_W4A16 ? mma::grouped_gemv_mma_kernel<MOE_W4A16>
                           : mma::grouped_gemv_mma_kernel<MOE_W4A4>;
     if ((st = set_smem(kern, mma::kSmemBytes)) != MOE_OK) return st;
-    kern<<<(unsigned)sms, mma::kThreads, mma::kSmemBytes, s>>>(p, ts_mma, maps.tlines);
+    kern<<<(unsigned)sms, mma::kThreads, mma::kSmemBytes, s>>>(p, ts_mma, maps.tlines,
+                                                               maps.tsf_lines);
     return launch_status();
   }
   void (*kern)(const Params, const CUtensorMap, const CUtensorMap);
