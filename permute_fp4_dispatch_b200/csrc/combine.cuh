@@ -23,6 +23,8 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     combine_kernel(const uint16_t *__restrict__ y, const float *__restrict__ rw,
                    const int64_t *__restrict__ ids, int32_t M, int32_t top_k, int32_t H,
                    int32_t E, float alpha, uint16_t *__restrict__ out) {
+  pdl_wait();
+  pdl_launch_dependents();
   const unsigned lane = lane_id();
   const int segs = (H + 255) / 256;
   const int64_t total = (int64_t)M * segs;

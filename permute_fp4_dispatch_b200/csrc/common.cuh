@@ -22,6 +22,17 @@ namespace moe {
 // Device error word (bits MOE_DEVERR_*), read by moe_get_device_error().
 __device__ unsigned int g_device_error;
 
+// Programmatic dependent launch.  pdl_wait(): block until the grids this
+// launch programmatically depends on have completed and their writes are
+// visible (a no-op when the launch has no such dependency); every kernel that
+// the library launches with the programmatic attribute calls it before
+// reading any input.  pdl_launch_dependents(): let the next such launch in the
+// stream be scheduled now (it still waits in its own pdl_wait()).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ void raise_device_error(unsigned int bit) {
   atomicOr(&g_device_error, bit);
 }

@@ -287,6 +287,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     int32_t *__restrict__ expert_ids,
                                     uint32_t *__restrict__ stats,
                                     uint32_t *__restrict__ scales_offset) {
+  pdl_wait();
+  pdl_launch_dependents();
   extern __shared__ __align__(16) uint8_t smem_raw[];
   const int WS = tiny_hist_stride(E);
   uint16_t *whist = reinterpret_cast<uint16_t *>(smem_raw);

@@ -47,6 +47,8 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
                           const int32_t *__restrict__ expert_ids,
                           const uint32_t *__restrict__ stats, uint8_t *__restrict__ recv,
                           int64_t capacity, int32_t stride, uint32_t *__restrict__ counts) {
+  pdl_wait();
+  pdl_launch_dependents();
   const unsigned lane = lane_id();
   if (blockIdx.x == 0) {  // recv_counts[e] from the CSR offsets
     for (int e = threadIdx.x; e < E; e += blockDim.x) counts[e] = 0u;

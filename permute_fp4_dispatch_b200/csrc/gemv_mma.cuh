@@ -196,6 +196,8 @@ template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemv_mma_kernel(const Params p, const int ts, const __grid_constant__ CUtensorMap tmap_w,
                             const __grid_constant__ CUtensorMap tmap_sf) {
+  pdl_wait();
+  pdl_launch_dependents();
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));

@@ -11,6 +11,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "combine.cuh"
 #include "common.cuh"
@@ -77,6 +78,30 @@ template <typename Kernel>
 moe_status_t set_smem(Kernel k, size_t bytes) {
   if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) !=
       cudaSuccess) {
+    cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
+// Launch with programmatic stream serialization: when the previous work in
+// the stream is a kernel, this grid may be scheduled before that kernel
+// finishes; the kernel's pdl_wait() holds it until the predecessor's writes
+// are visible.  Used for the kernels that call pdl_wait() first thing.
+template <typename... KArgs, typename... Args>
+moe_status_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                        cudaStream_t s, Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...) != cudaSuccess) {
     cudaGetLastError();
     return MOE_ERR_CUDA;
   }
@@ -327,10 +352,10 @@ moe_status_t moe_mask_and_create_indices(int64_t *routing_map, int32_t N, int32_
   if (st != MOE_OK) return st;
   const size_t smem = tiny_smem_bytes(E);
   if ((st = set_smem(mask_create_indices_tiny_kernel, smem)) != MOE_OK) return st;
-  mask_create_indices_tiny_kernel<<<1, kThreads, smem, s>>>(
-      routing_map, N, top_k, real_token_count, tp_rank, E, token_expert_order,
-      expert_start_indices, restore_token_order, expert_ids, expert_usage_stats, scales_offset);
-  return launch_status();
+  return launch_pdl(mask_create_indices_tiny_kernel, dim3(1), dim3(kThreads), smem, s, routing_map,
+                    N, top_k, real_token_count, tp_rank, E, token_expert_order,
+                    expert_start_indices, restore_token_order, expert_ids, expert_usage_stats,
+                    scales_offset);
 }
 
 // ------------------------------------------------------------------ step 3
@@ -373,11 +398,10 @@ moe_status_t moe_dispatch_mxfp4(const void *input_tokens, int32_t N, int32_t K, 
                              : seg == 4 ? moe::disp::dispatch_mxfp4_kernel<4>
                              : seg == 2 ? moe::disp::dispatch_mxfp4_kernel<2>
                                         : moe::disp::dispatch_mxfp4_kernel<1>;
-  kern<<<(unsigned)blocks, wpb * 32, 0, s>>>(
-      static_cast<const uint16_t *>(input_tokens), N, K, top_k, E, restore_token_order,
-      expert_start_indices, expert_ids, expert_usage_stats, recv_buf, recv_capacity,
-      (int32_t)moe_mxfp4_row_stride(K), recv_counts);
-  return launch_status();
+  return launch_pdl(kern, dim3((unsigned)blocks), dim3(wpb * 32), 0, s,
+                    static_cast<const uint16_t *>(input_tokens), N, K, top_k, E,
+                    restore_token_order, expert_start_indices, expert_ids, expert_usage_stats,
+                    recv_buf, recv_capacity, (int32_t)moe_mxfp4_row_stride(K), recv_counts);
 }
 
 // ------------------------------------------------------------------ step 4a
@@ -395,9 +419,8 @@ moe_status_t moe_quantize_activations_nvfp4(const void *x, int32_t M, int32_t K,
   const int64_t work = (int64_t)M * ((K + 255) / 256);
   int64_t blocks = (work + wpb - 1) / wpb;
   if (blocks > (int64_t)sms * 16) blocks = (int64_t)sms * 16;
-  moe::nvq::quant_act_nvfp4_kernel<<<(unsigned)blocks, wpb * 32, 0, s>>>(
-      static_cast<const uint16_t *>(x), M, K, act_global, xq, sfa);
-  return launch_status();
+  return launch_pdl(moe::nvq::quant_act_nvfp4_kernel, dim3((unsigned)blocks), dim3(wpb * 32), 0,
+                    s, static_cast<const uint16_t *>(x), M, K, act_global, xq, sfa);
 }
 
 moe_status_t moe_quantize_weights_nvfp4(const float *w, int32_t E, int32_t N, int32_t K,
@@ -491,9 +514,8 @@ moe_status_t moe_grouped_gemv_nvfp4(moe_gemv_mode_t mode, const void *act, const
         mode == MOE_W4A16 ? mma::grouped_gemv_mma_kernel<MOE_W4A16>
                           : mma::grouped_gemv_mma_kernel<MOE_W4A4>;
     if ((st = set_smem(kern, mma::kSmemBytes)) != MOE_OK) return st;
-    kern<<<(unsigned)sms, mma::kThreads, mma::kSmemBytes, s>>>(p, ts_mma, maps.tlines,
-                                                               maps.tsf_lines);
-    return launch_status();
+    return launch_pdl(kern, dim3((unsigned)sms), dim3(mma::kThreads), mma::kSmemBytes, s, p,
+                      ts_mma, maps.tlines, maps.tsf_lines);
   }
   void (*kern)(const Params, const CUtensorMap, const CUtensorMap);
   if (mode == MOE_W4A16)
@@ -503,8 +525,8 @@ moe_status_t moe_grouped_gemv_nvfp4(moe_gemv_mode_t mode, const void *act, const
     kern = maps.sf_tma ? tc::grouped_gemv_kernel<MOE_W4A4, true>
                        : tc::grouped_gemv_kernel<MOE_W4A4, false>;
   if ((st = set_smem(kern, tc::kSmemBytes)) != MOE_OK) return st;
-  kern<<<(unsigned)sms, tc::kThreads, tc::kSmemBytes, s>>>(p, maps.tw, maps.tsf);
-  return launch_status();
+  return launch_pdl(kern, dim3((unsigned)sms), dim3(tc::kThreads), tc::kSmemBytes, s, p, maps.tw,
+                    maps.tsf);
 }
 
 // ------------------------------------------------------------------ step 5
@@ -530,12 +552,11 @@ moe_status_t moe_combine(const void *expert_out, const float *router_weights,
   const uint16_t *y = static_cast<const uint16_t *>(expert_out);
   uint16_t *o = static_cast<uint16_t *>(output_tokens);
   if (epi == MOE_EPI_SCALE)
-    moe::comb::combine_kernel<MOE_EPI_SCALE><<<(unsigned)blocks, wpb * 32, 0, s>>>(
-        y, router_weights, topk_ids, M, top_k, H, E, alpha, o);
-  else
-    moe::comb::combine_kernel<MOE_EPI_IDENTITY><<<(unsigned)blocks, wpb * 32, 0, s>>>(
-        y, router_weights, topk_ids, M, top_k, H, E, alpha, o);
-  return launch_status();
+    return launch_pdl(moe::comb::combine_kernel<MOE_EPI_SCALE>, dim3((unsigned)blocks),
+                      dim3(wpb * 32), 0, s, y, router_weights, topk_ids, M, top_k, H, E, alpha,
+                      o);
+  return launch_pdl(moe::comb::combine_kernel<MOE_EPI_IDENTITY>, dim3((unsigned)blocks),
+                    dim3(wpb * 32), 0, s, y, router_weights, topk_ids, M, top_k, H, E, alpha, o);
 }
 
 }  // extern "C"

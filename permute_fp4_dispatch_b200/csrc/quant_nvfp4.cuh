@@ -43,6 +43,8 @@ __device__ __forceinline__ uint32_t encode_half_block(const float (&f)[8], float
 __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     quant_act_nvfp4_kernel(const uint16_t *__restrict__ x, int32_t M, int32_t K, float g,
                            uint8_t *__restrict__ xq, uint8_t *__restrict__ sfa) {
+  pdl_wait();
+  pdl_launch_dependents();
   const unsigned lane = lane_id();
   const int64_t segs = (K + 255) / 256;
   const int64_t total = (int64_t)M * segs;

@@ -98,6 +98,9 @@ class RoutingPipeline:
         self.expert_out = torch.zeros((N, top_k, N_out), dtype=torch.bfloat16, device=dev)
         # step 5
         self.output = torch.empty((N, N_out), dtype=torch.bfloat16, device=dev)
+        # timing events go on a side stream, so no event sits between two kernels
+        # of the main stream (which would cut their programmatic dependency)
+        self._timer = torch.cuda.Stream(device=dev)
 
     def host_inputs(self):
         """A pinned host byte buffer laid out like ``inputs`` and its typed
@@ -157,7 +160,8 @@ class RoutingPipeline:
 
     def run(self, stream=None, gemv_events=None, side_stream=None, x_ready=None):
         """All steps in order.  ``gemv_events`` = (start, end) CUDA events
-        recorded around the GEMV launch, for per-kernel timing.  With
+        recorded around the GEMV launch (from a side stream), for per-kernel
+        timing.  With
         ``side_stream``, the MXFP4 dispatch (whose buffer neither the GEMV nor
         the combine reads) runs there, forked after the GEMV and joined at the
         end, so it overlaps the combine instead of holding SMs the GEMV's
@@ -174,10 +178,10 @@ class RoutingPipeline:
         if self.gemv_mode == MOE_W4A4:
             self.quantize_activations(main)
         if gemv_events is not None:
-            gemv_events[0].record(main)
+            self._mark(main, gemv_events[0])
         self.gemv(main)
         if gemv_events is not None:
-            gemv_events[1].record(main)
+            self._mark(main, gemv_events[1])
         if forked:
             fork = torch.cuda.Event()
             fork.record(main)
@@ -188,6 +192,18 @@ class RoutingPipeline:
         self.combine(main)
         if forked:
             main.wait_event(join)
+        if gemv_events is not None:
+            timer_done = torch.cuda.Event()
+            timer_done.record(self._timer)
+            main.wait_event(timer_done)
+
+    def _mark(self, main, event):
+        """Record ``event`` once everything enqueued on ``main`` so far has run,
+        from the side timer stream."""
+        here = torch.cuda.Event()
+        here.record(main)
+        self._timer.wait_event(here)
+        event.record(self._timer)
 
     def launches_per_run(self) -> int:
         # mask + create_indices: one fused kernel up to 1024 slots, else mask and 1-2 kernels
