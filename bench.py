@@ -376,9 +376,11 @@ def run_ours(args, rank, world, local_rank):
     ms_gemv = float(np.mean(t_gemv))
 
     # end to end through the public API, host buffers: one CUDA graph per step
-    # holding the H2D copies of the step's inputs from pinned memory (routing
+    # holding the H2D copy of the step's inputs from pinned memory (routing
     # inputs first; the activations on a forked stream, overlapping mask and
-    # create_indices), the pipeline, and the D2H copy of the output
+    # create_indices) and the pipeline, whose combine stores the step's result
+    # straight into pinned host memory (a device-accessible pointer under
+    # unified addressing), so the result crosses PCIe without a separate copy
     e2e_ms = []
     h2d = h_in.numel()   # routing map, router weights, real_token_count, x (+ alignment gaps)
     d2h = h_out.numel() * 2
@@ -397,12 +399,14 @@ def run_ours(args, rank, world, local_rank):
         x_ready = torch.cuda.Event()
         x_ready.record(xcopy)
         pipe.run(cur, side_stream=side, x_ready=x_ready)
-        h_out.copy_(pipe.output, non_blocking=True)
 
+    dev_out = pipe.output
+    pipe.output = h_out                                   # the combine's output buffer
     with torch.cuda.stream(stream):
         e2e_step_ops()                                    # warm-up outside capture
         with torch.cuda.graph(e2e_graph, stream=stream):
             e2e_step_ops()
+    pipe.output = dev_out
     stream.synchronize()
     for i in range(args.warmup + args.steps):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -415,7 +419,10 @@ def run_ours(args, rank, world, local_rank):
         if i >= args.warmup:
             e2e_ms.append(e0.elapsed_time(e1))
     torch.cuda.synchronize()
-    # the host copy of the last step's output is the device result
+    # the result that reached the host is the device step's result
+    with torch.cuda.stream(stream):
+        graph.replay()
+    stream.synchronize()
     assert torch.equal(h_out.view(torch.int16), pipe.output.cpu().view(torch.int16))
     e2e_step = max_over_ranks(float(np.mean(e2e_ms)), world, dev)
 

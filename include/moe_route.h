@@ -258,6 +258,9 @@ MOE_API moe_status_t moe_grouped_gemv_nvfp4(moe_gemv_mode_t mode, const void *ac
 /* slots are never read), router_weights fp32 [M, top_k], topk_ids int64 */
 /* [M, top_k], output_tokens bf16 [M, H].  H (hidden_size) is the expert */
 /* output width.  Limits: H % 8 == 0, 16-byte aligned bf16 buffers.       */
+/* output_tokens may be pinned host memory (a device-accessible pointer   */
+/* under unified addressing): the result then reaches the host through   */
+/* the kernel's own stores, without a separate copy.                     */
 MOE_API moe_status_t moe_combine(const void *expert_out, const float *router_weights,
                          const int64_t *topk_ids, int32_t M, int32_t top_k, int32_t H, int32_t E,
                          moe_epilogue_t epi, float alpha, void *output_tokens, cudaStream_t s);

@@ -405,6 +405,19 @@ def test_combine_one_hot_is_exact():
     np.testing.assert_array_equal(host_bf16_bits(out), y[np.arange(8), sel])
 
 
+def test_combine_into_pinned_host_memory():
+    """output_tokens may be pinned host memory: same bytes as a device buffer."""
+    cfg = wl.config("decode_30b_a3b")
+    y, w = dev(wl.expert_outputs_bf16(cfg)), dev(wl.router_weights(cfg))
+    ids = dev(wl.routing(cfg))
+    out_dev = torch.empty((cfg.N, cfg.N_out), dtype=torch.bfloat16, device="cuda")
+    out_host = torch.full((cfg.N, cfg.N_out), 7.0, dtype=torch.bfloat16).pin_memory()
+    moe.moe_combine(y, w, ids, cfg.N, cfg.top_k, cfg.N_out, cfg.E, 1, 1.0, out_dev)
+    moe.moe_combine(y, w, ids, cfg.N, cfg.top_k, cfg.N_out, cfg.E, 1, 1.0, out_host)
+    torch.cuda.synchronize()
+    assert torch.equal(out_host.view(torch.int16), out_dev.cpu().view(torch.int16))
+
+
 # ------------------------------------------------------------------ boundary
 def test_invalid_arguments_launch_nothing():
     with pytest.raises(moe.MoeError) as e:
