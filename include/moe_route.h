@@ -255,7 +255,7 @@ MOE_API moe_status_t moe_grouped_gemv_nvfp4(moe_gemv_mode_t mode, const void *ac
 /*   output_tokens[t, h] = bf16( epi( sum_{j: 0<=id<E} w[t,j]*y[t,j,h] ) ) */
 /* fp32 accumulation in slot order; a row with no routed slot gives      */
 /* epi(0).  expert_out bf16 [M, top_k, H] (the GEMV output; unrouted     */
-/* slots are never read), router_weights fp32 [M, top_k], topk_ids int64 */
+/* slots are never used), router_weights fp32 [M, top_k], topk_ids int64 */
 /* [M, top_k], output_tokens bf16 [M, H].  H (hidden_size) is the expert */
 /* output width.  Limits: H % 8 == 0, 16-byte aligned bf16 buffers.       */
 /* output_tokens may be pinned host memory (a device-accessible pointer   */

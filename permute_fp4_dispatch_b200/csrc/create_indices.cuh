@@ -301,14 +301,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int S = N * top_k;
   const unsigned lt = (1u << lane) - 1u;
 
-  // step 1 + key: one load per slot
+  // step 1 + key: one load per slot, issued together with the count's
   int key = -1;
+  const int64_t id = p < S ? ids[p] : -1;
+  const int64_t real = *real_count;
   if (p < S) {
     const int row = p / top_k;
-    if ((int64_t)row + (int64_t)tp_rank * N >= (int64_t)*real_count) {
+    if ((int64_t)row + (int64_t)tp_rank * N >= real) {
       ids[p] = -1;
     } else {
-      const int64_t id = ids[p];
       key = (id >= 0 && id < E) ? (int)id : -1;
     }
   }
