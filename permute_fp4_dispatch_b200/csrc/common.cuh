@@ -58,18 +58,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 // ------------------------------------------------------------------ FP4 / FP8 conversions
-// Two fp32 -> one byte of E2M1 codes (RNE, saturating); `lo` goes to the low
-// nibble.  The PTX instruction stores its first source in the upper nibble.
-__device__ __forceinline__ uint32_t e2m1x2_from_f32(float lo, float hi) {
-  uint32_t out;
-  asm("{\n\t.reg .b8 q;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 q, %1, %2;\n\t"
-      "cvt.u32.u8 %0, q;\n\t}"
-      : "=r"(out)
-      : "f"(hi), "f"(lo));
-  return out;
-}
-
 // Eight fp32 -> four bytes (element 0 in the low nibble of byte 0).
 __device__ __forceinline__ uint32_t e2m1x8_from_f32(const float *v) {
   uint32_t out;
@@ -201,17 +189,6 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
   }
 }
 
-// Global -> shared bulk copy on the TMA engine, completing on `bar`.
-// dst, src 16-byte aligned; bytes a multiple of 16.
-__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes,
-                                         uint64_t *bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
-          "r"(smem_addr(dst)),
-      "l"(src), "r"(bytes), "r"(smem_addr(bar))
-      : "memory");
-}
-
 // L2 policy for data read exactly once (streamed weights).
 __device__ __forceinline__ uint64_t l2_evict_first_policy() {
   uint64_t pol;
@@ -250,13 +227,6 @@ __device__ __forceinline__ void prefetch_tmap(const void *tmap) {
 // 4-byte asynchronous copy global -> shared (both 4-byte aligned).
 __device__ __forceinline__ void cp_async4(void *dst, const void *src) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_addr(dst)), "l"(src)
-               : "memory");
-}
-
-// 16-byte asynchronous copy global -> shared, bypassing L1 (both 16-byte
-// aligned), without an L2 cache-policy operand.
-__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)), "l"(src)
                : "memory");
 }
 

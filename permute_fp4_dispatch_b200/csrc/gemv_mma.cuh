@@ -196,8 +196,6 @@ template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemv_mma_kernel(const Params p, const int ts, const __grid_constant__ CUtensorMap tmap_w,
                             const __grid_constant__ CUtensorMap tmap_sf) {
-  pdl_wait();
-  pdl_launch_dependents();
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -213,6 +211,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = (int)lane_id();
+  // set-up that reads no input runs before the wait for the previous grid
+  if (threadIdx.x == 0) {
+    // one arrival with the byte count of the stage's two TMA boxes
+    for (int i = 0; i < kCW * kSlots; ++i) mbar_init(&full[i], 1u);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (lane == 0) {
+    prefetch_tmap(&tmap_w);
+    prefetch_tmap(&tmap_sf);
+  }
+  pdl_wait();
+  pdl_launch_dependents();
   const int N = p.N, K = p.K;
   const int RB = (N + 15) / 16;
   const uint32_t A = p.stats[1];
@@ -234,12 +245,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       s_range[1] = u1;
     }
   }
-  if (threadIdx.x == 0) {
-    // one arrival with the byte count of the stage's two TMA boxes
-    for (int i = 0; i < kCW * kSlots; ++i) mbar_init(&full[i], 1u);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
   __syncthreads();
 
   const uint32_t u_begin = s_range[0], u_end = s_range[1];
@@ -251,10 +256,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *sring = smem + kOffSF + (size_t)warp * kSlots * kStageSF;
   uint64_t *wfull = full + warp * kSlots;
   const uint64_t policy = l2_evict_first_policy();
-  if (lane == 0) {
-    prefetch_tmap(&tmap_w);
-    prefetch_tmap(&tmap_sf);
-  }
 
   // ---- producer side of this warp's pipeline: the next (round, stage) of its blocks
   RoundWalk piter;
