@@ -58,6 +58,17 @@ def parse_args():
     return ap.parse_args()
 
 
+METRIC = "routed token-expert pairs/s end-to-end at 1 B200"
+
+
+def workload_config(cfg, mode: str, routed_pairs: int, active_experts: int) -> dict:
+    """The config keys both arms report for a workload."""
+    return {"workload": cfg.name, "N": cfg.N, "real_token_count": cfg.real, "K": cfg.K,
+            "E": cfg.E, "top_k": cfg.top_k, "N_out": cfg.N_out, "mode": mode,
+            "routed_pairs": routed_pairs, "active_experts": active_experts,
+            "parallelism": "replicas"}
+
+
 def max_over_ranks(value: float, world: int, device="cpu") -> float:
     """The largest value over the ranks (a replica job's time is its slowest
     replica's); with one rank, the value itself."""
@@ -218,6 +229,13 @@ def oracle_setup(cfg, mode, n_tokens):
     return x, ids, rw, tokens, wq, sfw, gw, experts
 
 
+def routed_pairs_and_active(cfg):
+    """Routed pairs and active experts of the whole workload, from the oracle."""
+    import oracle
+    idx = oracle.create_indices(oracle.mask_padding(wl.routing(cfg), cfg.real), cfg.E)
+    return int(idx["expert_start_indices"][-1]), int(idx["expert_usage_stats"][1])
+
+
 def cpu_cores() -> int:
     try:
         return len(os.sched_getaffinity(0))
@@ -255,6 +273,7 @@ def run_reference(args, rank, world):
     n_tokens = int(max(1, min(args.cpu_sample_tokens, budget / max(t_token, 1e-6))))
     setup = oracle_setup(cfg, mode, n_tokens)
     tokens = setup[3]
+    full_idx = routed_pairs_and_active(cfg)
     for _ in range(args.warmup):
         oracle_sample_step(cfg, mode, *setup[:3], tokens, *setup[4:])
     times = []
@@ -266,13 +285,12 @@ def run_reference(args, rank, world):
     dt = float(np.mean(times))
     value = pairs / dt
     line = {
-        "impl": "reference", "metric": "routed token-expert pairs/s end-to-end",
+        "impl": "reference", "metric": METRIC,
         "value": value, "unit": "routed pairs/s", "n_gpus": args.gpus, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": cfg.name, "N": cfg.N, "real_token_count": cfg.real, "K": cfg.K,
-                   "E": cfg.E, "top_k": cfg.top_k, "N_out": cfg.N_out, "mode": mode,
-                   "sample_tokens": int(len(tokens)), "parallelism": "replicas"},
+        "config": dict(workload_config(cfg, mode, full_idx[0], full_idx[1]),
+                       sample_tokens=int(len(tokens))),
         "e2e": {"value": value, "unit": "routed pairs/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
         "cpu_baseline": {"value": value, "unit": "routed pairs/s", "cores": 1, "kind": "oracle",
@@ -431,19 +449,17 @@ def run_ours(args, rank, world, local_rank):
     gemv_gbs = bytes_["grouped_gemv"] / (ms_gemv * 1e-3) / 1e9
     total_bytes = sum(bytes_.values())
     line = {
-        "metric": "routed token-expert pairs/s end-to-end at 1 B200",
+        "metric": METRIC,
         "value": job_rate(R, world, ms_step),
         "unit": "routed pairs/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "fp4xbf16->f32" if mode == "w4a16" else "fp4xfp4->f32",
         "data": "synthetic (seeded; weights N(0,0.02) quantised to NVFP4 on device)",
-        "config": {"workload": cfg.name, "N": cfg.N, "real_token_count": cfg.real, "K": cfg.K,
-                   "E": cfg.E, "top_k": cfg.top_k, "N_out": cfg.N_out, "mode": mode,
-                   "routed_pairs": R, "active_experts": A,
-                   "l2": "flushed before every step (512 MiB memset outside the timed events)",
-                   "graph": "one CUDA graph per step (dispatch on a forked stream after the GEMV, beside the combine)",
-                   "parallelism": "replicas"},
+        "config": dict(workload_config(cfg, mode, R, A),
+                       l2="flushed before every step (512 MiB memset outside the timed events)",
+                       graph="one CUDA graph per step (dispatch on a forked stream after the "
+                             "GEMV, beside the combine)"),
         "roofline": {"kernel": "grouped_gemv_nvfp4", "bound": "hbm", "achieved": gemv_gbs,
                      "peak": peak, "unit": "GB/s", "frac": gemv_gbs / peak,
                      "traffic": profiled_traffic(cfg.name),
