@@ -220,6 +220,13 @@ __device__ __forceinline__ void tma_load_4d(void *dst, const void *tmap, int x, 
       : "memory");
 }
 
+// L2 prefetch hint for [src, src + bytes): src 16-byte aligned, bytes a
+// multiple of 16.  Only warms L2, so it is safe on memory another grid may
+// still be writing (L2 is where every write lands).
+__device__ __forceinline__ void prefetch_l2_bulk(const void *src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ void prefetch_tmap(const void *tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
 }

@@ -16,7 +16,7 @@ struct Params {
   const void *act;          // W4A16: bf16 [M, K]; W4A4: u8 [M, K/2]
   const uint8_t *sfa;       // W4A4: [M, K/16]
   float g_a;
-  int32_t top_k;
+  int32_t M, top_k;
   const uint8_t *w;         // [E, N, K/2]
   const uint8_t *sfw;       // [E, N, K/16]
   const float *w_global;    // [E] or null
@@ -85,17 +85,26 @@ struct RoundIter {
   }
 };
 
+// floor(a * b / c) for a quotient below 2^32, dividing in 32 bits whenever the
+// product fits (a 64-bit division is a long software sequence, and one
+// thread computes the partition while the CTA waits).
+__device__ __forceinline__ uint32_t muldiv(uint32_t a, uint32_t b, uint32_t c) {
+  const uint64_t ab = (uint64_t)a * b;
+  return (ab >> 32) == 0 ? (uint32_t)ab / c : (uint32_t)(ab / c);
+}
+
 // This CTA's share [u0, u1) of the U units, cut at round boundaries: every
 // pass (RB units) splits into ceil(RB / rbk) rounds of up to rbk blocks, and
 // the grid shares the rounds evenly, so no round is split between CTAs and a
 // CTA's warps never face a partial round in the middle of a pass.
 __device__ __forceinline__ void cta_round_range(uint32_t U, int RB, int rbk, uint32_t &u0,
                                                 uint32_t &u1) {
-  const uint64_t R = (uint64_t)((RB + rbk - 1) / rbk);
-  const uint64_t T = (uint64_t)(U / (uint32_t)RB) * R;
-  const uint64_t r0 = T * blockIdx.x / gridDim.x, r1 = T * (blockIdx.x + 1) / gridDim.x;
-  u0 = (uint32_t)((r0 / R) * (uint64_t)RB + (r0 % R) * (uint64_t)rbk);
-  u1 = (uint32_t)((r1 / R) * (uint64_t)RB + (r1 % R) * (uint64_t)rbk);
+  const uint32_t R = (uint32_t)((RB + rbk - 1) / rbk);
+  const uint32_t T = U / (uint32_t)RB * R;  // rounds in all; T <= U
+  const uint32_t r0 = muldiv(T, blockIdx.x, gridDim.x);
+  const uint32_t r1 = muldiv(T, blockIdx.x + 1, gridDim.x);
+  u0 = r0 / R * (uint32_t)RB + r0 % R * (uint32_t)rbk;
+  u1 = r1 / R * (uint32_t)RB + r1 % R * (uint32_t)rbk;
 }
 
 // As cta_round_range, but when the passes (U / RB of them) are no more than
@@ -105,20 +114,21 @@ __device__ __forceinline__ void cta_round_range(uint32_t U, int RB, int rbk, uin
 // passes.
 __device__ __forceinline__ void cta_pass_range(uint32_t U, int RB, int rbk, uint32_t &u0,
                                                uint32_t &u1) {
-  const uint64_t P = U / (uint32_t)RB, G = gridDim.x, b = blockIdx.x;
+  const uint32_t P = U / (uint32_t)RB, G = gridDim.x, b = blockIdx.x;
   if (P == 0 || P > G) {
     cta_round_range(U, RB, rbk, u0, u1);
     return;
   }
-  const uint64_t pass = b * P / G;
-  const uint64_t first = (pass * G + P - 1) / P;        // first CTA of the pass
-  const uint64_t count = ((pass + 1) * G + P - 1) / P - first;
-  const uint64_t i = b - first;
-  const uint64_t R = (uint64_t)((RB + rbk - 1) / rbk);
-  const uint64_t r0 = R * i / count, r1 = R * (i + 1) / count;
-  const uint64_t base = pass * (uint64_t)RB;
-  u0 = (uint32_t)(base + min((uint64_t)RB, r0 * (uint64_t)rbk));
-  u1 = (uint32_t)(base + min((uint64_t)RB, r1 * (uint64_t)rbk));
+  // P <= G, and G (one CTA per SM) is below 2^16, so every product here fits 32 bits
+  const uint32_t pass = b * P / G;
+  const uint32_t first = (pass * G + P - 1) / P;        // first CTA of the pass
+  const uint32_t count = ((pass + 1) * G + P - 1) / P - first;
+  const uint32_t i = b - first;
+  const uint32_t R = (uint32_t)((RB + rbk - 1) / rbk);
+  const uint32_t r0 = muldiv(R, i, count), r1 = muldiv(R, i + 1, count);
+  const uint32_t base = pass * (uint32_t)RB;
+  u0 = base + (uint32_t)min((uint64_t)RB, (uint64_t)r0 * (uint32_t)rbk);
+  u1 = base + (uint32_t)min((uint64_t)RB, (uint64_t)r1 * (uint32_t)rbk);
 }
 
 __device__ __forceinline__ uint32_t bcast_lo(uint32_t h) { return __byte_perm(h, h, 0x1010); }

@@ -60,6 +60,7 @@ constexpr int kGroupStageBytes = 8 * kKS * 2;  // fp16 tile of one 8-token group
 constexpr int kActBytes = 64 * 1024;
 constexpr int kStagingBytes = kCW * kMaxTS * 16 * 2;
 constexpr uint64_t kDrainLimitNs = 100000000ull;  // 100 ms
+constexpr uint64_t kActPrefetchMax = 8u << 20;     // activations prefetched into L2 up to 8 MiB
 // 16-byte activation slices per thread in a pass setup: the tile holds
 // kActBytes / 16 slices, spread over the CTA.
 constexpr int kSetupTasks = kActBytes / 16 / kThreads;
@@ -222,6 +223,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tmap_w);
     prefetch_tmap(&tmap_sf);
   }
+  if (MODE == MOE_W4A16 && threadIdx.x == 32) {
+    // The bf16 activations are an input of the step, not of the grid this
+    // launch waits for: every CTA pulls its share of them into L2 while it
+    // waits, so the pass set-up finds them there.
+    const uint32_t bytes = (uint32_t)p.M * (uint32_t)p.K * 2u;  // K % 64 == 0
+    if ((uint64_t)p.M * p.K * 2u <= kActPrefetchMax) {
+      const uint32_t chunk = ((bytes + gridDim.x - 1) / gridDim.x + 15u) & ~15u;
+      const uint32_t end = min(bytes, chunk * (blockIdx.x + 1));
+      for (uint32_t off = chunk * blockIdx.x; off < end; off += 16384u)
+        prefetch_l2_bulk(static_cast<const uint8_t *>(p.act) + off, min(16384u, end - off));
+    }
+  }
   pdl_wait();
   pdl_launch_dependents();
   const int N = p.N, K = p.K;
@@ -311,21 +324,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---- new (expert, pass): build its fp16 activation tile for the whole K.
       // The loads (token order, then activation slices) are issued before the
       // barrier that frees the previous tile, so their latency overlaps it.
+      // Task b of a thread is slice kk of token tau, task = b * kThreads + tid =
+      // tau * per_tok + kk.  per_tok is a multiple of 32, so tau is the same
+      // across a warp, and lane j of every warp holds the row of token j.
       const int per_tok = kpad / 8;  // 8-column slices per token
       const int ntask = r.ntok * per_tok;  // at most kSetupTasks * kThreads
+      const int tau0 = (int)threadIdx.x / per_tok, kk0 = (int)threadIdx.x - tau0 * per_tok;
       uint4 v[kSetupTasks];
       uint32_t sv[kSetupTasks];
-      uint32_t my_pair = 0;
-      if ((int)threadIdx.x < r.ntok) my_pair = __ldg(p.order + r.tok0 + threadIdx.x);
+      uint32_t my_pair = 0, my_row = 0;
+      if (lane < r.ntok) {
+        my_pair = __ldg(p.order + r.tok0 + lane);
+        my_row = my_pair / (uint32_t)p.top_k;
+      }
+      int tau = tau0, kk = kk0;
 #pragma unroll
       for (int b = 0; b < kSetupTasks; ++b) {
         const int task = b * kThreads + (int)threadIdx.x;
+        const int64_t m = (int64_t)__shfl_sync(0xFFFFFFFFu, my_row, tau & 31);
+        const int k = kk * 8;
         v[b] = make_uint4(0u, 0u, 0u, 0u);
         sv[b] = 0u;
         if (task < ntask) {
-          const int tau = task / per_tok;
-          const int k = (task % per_tok) * 8;
-          const int64_t m = (int64_t)(__ldg(p.order + r.tok0 + tau) / (uint32_t)p.top_k);
           if (k < K) {
             if (MODE == MOE_W4A16) {
               v[b] = ldg_nc_v4(static_cast<const uint16_t *>(p.act) + m * K + k);
@@ -336,6 +356,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
+        for (kk += kThreads; kk >= per_tok; kk -= per_tok) ++tau;
       }
       if (!primed) {
         for (int st = 0; st < kSlots; ++st) produce();
@@ -345,12 +366,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       ng = (r.ntok + 7) / 8;
       if ((int)threadIdx.x < r.ntok) s_pair[threadIdx.x] = my_pair;
       unsigned range_bad = 0;
+      tau = tau0;
+      kk = kk0;
 #pragma unroll
       for (int b = 0; b < kSetupTasks; ++b) {
         const int task = b * kThreads + (int)threadIdx.x;
+        const int tk = tau, k = kk * 8;
+        for (kk += kThreads; kk >= per_tok; kk -= per_tok) ++tau;
         if (task >= ntask) continue;
-        const int tau = task / per_tok;
-        const int k = (task % per_tok) * 8;
         uint4 hv = make_uint4(0u, 0u, 0u, 0u);
         if (k < K) {
           if (MODE == MOE_W4A16) {
@@ -375,9 +398,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             hv.w = hmul2(q3, sc);
           }
         }
-        // columns [k, k + 8): stage c, line lt, MMA pair m of lane (tau % 8, lt)
-        const int c = k / kKS, kk = k % kKS, lt = kk / 256, m = (kk % 256) / 8;
-        act[act_index(c, ng, tau / 8, m, (tau & 7) * 4 + lt)] = hv;
+        // columns [k, k + 8): stage c, line lt, MMA pair m of lane (tk % 8, lt)
+        const int c = k / kKS, kc = k % kKS, lt = kc / 256, m = (kc % 256) / 8;
+        act[act_index(c, ng, tk / 8, m, (tk & 7) * 4 + lt)] = hv;
       }
       if (MODE == MOE_W4A16 && range_bad) raise_device_error(MOE_DEVERR_ACT_RANGE);
       named_bar_sync(1, kThreads);

@@ -484,6 +484,7 @@ moe_status_t moe_grouped_gemv_nvfp4(moe_gemv_mode_t mode, const void *act, const
   p.act = act;
   p.sfa = sfa;
   p.g_a = act_global;
+  p.M = M;
   p.top_k = top_k;
   p.w = w;
   p.sfw = sfw;
