@@ -5,7 +5,7 @@ the library's kernels do all the work.
     pipe.quantize_weights(w_f32_expert_slices)      # offline, once
     pipe.x.copy_(...); pipe.routing_map.copy_(...); pipe.router_weights.copy_(...)
     pipe.real_token_count.fill_(real)
-    pipe.run()                                      # mask + indices -> dispatch || GEMV -> combine
+    pipe.run()                                      # mask + indices -> GEMV (|| dispatch) -> combine
     pipe.output                                     # bf16 [N, N_out]
 
 Every buffer is allocated once at construction, so ``run`` allocates
@@ -44,6 +44,11 @@ def _arena_views(buf: torch.Tensor, entries):
 
 
 class RoutingPipeline:
+    # where run() forks the MXFP4 dispatch onto side_stream: "routing" (after
+    # mask + create_indices, beside the GEMV, on SMs its CTAs leave free) or
+    # "gemv" (after the GEMV, beside the combine)
+    dispatch_fork = "routing"
+
     def __init__(self, N: int, K: int, E: int, top_k: int, N_out: int, mode: str = "w4a16",
                  epilogue: str = "none", alpha: float = 1.0, tp_rank: int = 0,
                  act_global: float = 1.0, device: str | torch.device = "cuda",
@@ -101,6 +106,11 @@ class RoutingPipeline:
         # timing events go on a side stream, so no event sits between two kernels
         # of the main stream (which would cut their programmatic dependency)
         self._timer = torch.cuda.Stream(device=dev)
+        # recorded on the side stream before a dispatch forked after the routing
+        # kernel: a graph's event-record node there turns the dispatch's
+        # programmatic dependency into a plain one, so its CTAs do not take SMs
+        # before the GEMV's.  Kept alive with the pipeline (captured graphs use it).
+        self._dispatch_marker = torch.cuda.Event(external=True)
 
     def host_inputs(self):
         """A pinned host byte buffer laid out like ``inputs`` and its typed
@@ -161,18 +171,33 @@ class RoutingPipeline:
     def run(self, stream=None, gemv_events=None, side_stream=None, x_ready=None):
         """All steps in order.  ``gemv_events`` = (start, end) CUDA events
         recorded around the GEMV launch (from a side stream), for per-kernel
-        timing.  With
-        ``side_stream``, the MXFP4 dispatch (whose buffer neither the GEMV nor
-        the combine reads) runs there, forked after the GEMV and joined at the
-        end, so it overlaps the combine instead of holding SMs the GEMV's
-        persistent CTAs need.  ``x_ready`` (a CUDA event) holds back the steps
-        that read the activations -- dispatch, activation quantisation, GEMV --
-        until x has arrived; mask and create_indices run before it."""
+        timing.  With ``side_stream``, the MXFP4 dispatch (whose buffer neither
+        the GEMV nor the combine reads) runs there and joins at the end.  By
+        default (``dispatch_fork = "routing"``) it forks right after mask +
+        create_indices behind an event-record node, so it starts only once the
+        routing kernel is done: the GEMV's CTAs, launched early by the
+        programmatic dependency, hold the SMs first, and the dispatch runs on
+        the SMs they leave free, finishing before the GEMV does.  With
+        ``"gemv"`` it forks after the GEMV, beside the combine.  ``x_ready`` (a
+        CUDA event) holds back the steps that read the activations --
+        dispatch, activation quantisation, GEMV -- until x has arrived; mask
+        and create_indices run before it."""
         main = stream if stream is not None else torch.cuda.current_stream()
         self.mask_and_create_indices(main)
+        forked = self.dispatch and side_stream is not None
+        early = forked and self.dispatch_fork == "routing"
+        if early:
+            fork = torch.cuda.Event()
+            fork.record(main)
+            side_stream.wait_event(fork)
+            if x_ready is not None:
+                side_stream.wait_event(x_ready)
+            self._dispatch_marker.record(side_stream)
+            self.dispatch_mxfp4(side_stream)
+            join = torch.cuda.Event()
+            join.record(side_stream)
         if x_ready is not None:
             main.wait_event(x_ready)
-        forked = self.dispatch and side_stream is not None
         if self.dispatch and not forked:
             self.dispatch_mxfp4(main)
         if self.gemv_mode == MOE_W4A4:
@@ -182,7 +207,7 @@ class RoutingPipeline:
         self.gemv(main)
         if gemv_events is not None:
             self._mark(main, gemv_events[1])
-        if forked:
+        if forked and not early:
             fork = torch.cuda.Event()
             fork.record(main)
             side_stream.wait_event(fork)
