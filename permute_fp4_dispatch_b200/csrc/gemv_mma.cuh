@@ -7,10 +7,13 @@
 // At decode batch sizes the weight stream is the roofline and the
 // tensor-core work per weight is tiny (8-16 tokens), so this variant keeps
 // the tensor cores fed from registers and spends its effort on the stream:
-//   * Work partition shared with the tensor-memory variant: (active expert,
-//     pass, 16-row block) units in equal contiguous ranges per persistent
-//     CTA, rounds of up to 16 blocks of one (expert, pass); warp w owns block
-//     w of every round.
+//   * Work partition over (active expert, pass, 16-row block) units: when
+//     the passes are no more than the persistent CTAs, every CTA takes part
+//     of exactly one pass (cta_pass_range), else equal contiguous ranges cut
+//     at round boundaries; rounds of up to 16 blocks of one (expert, pass),
+//     warp w owns block w of every round.  The CTA computes its range once,
+//     after each CTA has pulled its slice of the bf16 activations into L2
+//     while waiting for the routing kernel (programmatic launch).
 //   * Every warp runs its own one-stage pipeline, with no producer warp and
 //     no cross-warp waits inside a pass; sixteen warps (four per scheduler)
 //     hide each other's load and dependency latencies.  A stage is 16 rows x
@@ -25,9 +28,9 @@
 //     4 * row + line, so the swizzle key is (row & 1) * 4 + line and the eight
 //     lanes of one shared-memory phase (rows g, g + 1) hit eight distinct
 //     16-byte bank groups.
-//   * When a CTA starts a new (expert, pass), the 8 warps convert that pass's
-//     activation rows once, for the whole K, into an fp16 tile laid out in
-//     mma fragment order; every round of the pass reuses it.  W4A16: plain
+//   * When a CTA starts a new (expert, pass), its 16 warps convert that
+//     pass's activation rows once, for the whole K, into an fp16 tile laid
+//     out in mma fragment order; every round of the pass reuses it.  W4A16: plain
 //     bf16 -> fp16 (exact for 2^-14 <= |x| <= 65504, MOE_DEVERR_ACT_RANGE
 //     beyond); W4A4: E2M1 x E4M3 products, exact in fp16.
 //   * Each lane dequantises its codes in registers (hardware E2M1 -> f16x2

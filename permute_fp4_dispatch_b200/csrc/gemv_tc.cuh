@@ -7,12 +7,13 @@
 // [M, top_k, N]).  For each routed pair p with expert e:
 //     out[p, n] = bf16( g_w[e] * g_a * sum_k a(p/top_k, k) * w(e, n, k) ).
 //
-// Design (decode-first; the FP4 weight stream is the roofline):
+// Design (taken when experts hold more tokens than a decode pass; the FP4
+// weight stream and its dequantisation bound it):
 //   * Work is expert-major: an active expert's pairs (CSR from
 //     moe_create_indices) are taken in passes of up to kTS = 64 tokens and
 //     each pass sweeps the expert's N rows in 16-row blocks.  The flat list of
-//     (expert, pass, row block) units is split into equal contiguous ranges,
-//     one per persistent CTA (grid = SM count).  Consecutive blocks of one
+//     (expert, pass, row block) units is split into equal contiguous ranges
+//     cut at round boundaries, one per persistent CTA (grid = SM count).  Consecutive blocks of one
 //     (expert, pass) form a round of up to 128 rows: one tcgen05 MMA tile
 //     (M = 128 weight rows, N = tokens rounded up to 16, fp32 in TMEM).
 //   * Warp roles (10 warps):
