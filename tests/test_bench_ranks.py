@@ -57,3 +57,29 @@ def test_single_rank_is_identity():
     import bench
     assert bench.max_over_ranks(2.0, 1) == 2.0
     assert bench.job_rate(10, 1, 1.0) == pytest.approx(10000.0)
+
+
+def test_reference_arm_line_matches_the_cuda_arm_contract():
+    """The reference arm (the oracle on host cores) prints one JSON line with the
+    CUDA arm's metric, unit, direction and workload keys, plus its own
+    cpu_baseline and a zero-copy e2e."""
+    import json
+    import subprocess
+    import bench
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--config", "tiny", "--steps", "1", "--warmup", "1"],
+                         capture_output=True, text=True, timeout=600, check=True).stdout
+    lines = [json.loads(l) for l in out.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    line = lines[0]
+    assert line["impl"] == "reference"
+    assert line["metric"] == bench.METRIC
+    assert line["unit"] == "routed pairs/s" and line["higher_is_better"] is True
+    assert line["value"] > 0 and line["steps"] == 1 and line["warmup"] == 1
+    cfg = bench.wl.config("tiny")
+    expect = bench.workload_config(cfg, cfg.modes[0], *bench.routed_pairs_and_active(cfg))
+    for k, v in expect.items():
+        assert line["config"][k] == v, k
+    assert line["e2e"] == {"value": line["value"], "unit": line["unit"],
+                           "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 1
