@@ -7,16 +7,19 @@
 One step = the whole hot path over one batch: mask -> create_indices ->
 MXFP4 dispatch -> [NVFP4 activation quantisation] -> grouped NVFP4 GEMV ->
 combine, replayed as one CUDA graph.  Inputs are resident in HBM when the
-timed region starts; L2 is flushed (a 512 MiB memset, outside the timed
-events) before every timed step.  Metric: routed token-expert pairs per
-second, whole job.  With N > 1 (torchrun) every rank runs an independent
+timed region starts; L2 is flushed before every timed step (a 512 MiB memset
+outside the timed events; ``--flush write+read`` adds a 512 MiB read so the
+step does not write back the flush's own dirty lines).  Metric: routed
+token-expert pairs per second, whole job.  With N > 1 (torchrun) every rank runs an independent
 replica of the workload (weak scaling; the path has no exchange step).
 
 Also reported: the grouped GEMV's achieved HBM bandwidth against the
-measured copy bandwidth (roofline), the pipeline's algorithmic-byte
-fraction, an end-to-end figure through the public API with host buffers,
-SM clocks sampled during the timed region, and the CPU oracle timed on a
-bounded sample of the same workload (rank 0, N = 1).
+measured copy bandwidth (roofline), every kernel's time and HBM fraction,
+the pipeline's algorithmic-byte fraction, an end-to-end figure through the
+public API with host buffers, SM clocks sampled during the timed region, the
+CPU oracle timed on a bounded sample of the same workload (rank 0, N = 1),
+and under "workloads" the same figures for the other synthetic workloads
+(tiny, decode large-expert, prefill index stress, gpt-oss-shaped W4A4).
 
 ``--impl reference`` times the CPU oracle itself as the reference arm.
 """
@@ -55,6 +58,10 @@ def parse_args():
     ap.add_argument("--config", default="decode_30b_a3b", choices=sorted(wl.CONFIGS))
     ap.add_argument("--cpu-sample-tokens", type=int, default=48)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="time the headline workload only")
+    ap.add_argument("--flush", choices=["write", "write+read"], default="write",
+                    help="how L2 is flushed between timed steps")
     return ap.parse_args()
 
 
@@ -86,13 +93,17 @@ def job_rate(units_per_rank: int, world: int, ms: float) -> float:
     return world * units_per_rank / (ms * 1e-3)
 
 
-def measured_peaks():
+def measured_peaks() -> dict:
+    """HBM copy bandwidth and dense bf16 tensor throughput measured on this
+    pool's B200s (MEASURED_PEAKS.json), else the recipe's fallback figures."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         with open(p) as f:
             d = json.load(f)
-        return float(d["hbm_gbs"]), "MEASURED_PEAKS.json hbm_gbs (of measured)"
-    return 6650.0, "profiling-recipe fallback 6.65 TB/s (of fallback)"
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "source": "MEASURED_PEAKS.json hbm_gbs / bf16_tflops (of measured)"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0,
+            "source": "profiling-recipe fallback 6.65 TB/s, 1.59 PFLOP/s (of fallback)"}
 
 
 def profiled_traffic(workload: str):
@@ -301,106 +312,160 @@ def run_reference(args, rank, world):
 
 
 # ------------------------------------------------------------------ our arm
-def run_ours(args, rank, world, local_rank):
+# which entries of the byte model each launch of a step accounts for
+KERNEL_BYTES = {"mask+create_indices": ("mask", "create_indices")}
+OTHER_WORKLOADS = ("tiny", "decode_large_expert", "prefill_index_stress", "gpt_oss_120b_w4a4")
+WORKLOAD_STEPS_CAP = 20    # timed steps per workload beyond the headline one
+
+
+def dense_flops(cfg, R: int) -> int:
+    """2 * R * N_out * K: the GEMV's multiply-adds over the routed pairs."""
+    return 2 * R * cfg.N_out * cfg.K
+
+
+class L2Flush:
+    """Between timed steps: write a buffer larger than L2, which evicts every
+    line of the step's inputs and outputs; mode "write+read" then reads
+    another one, so that the next step starts with clean lines of unrelated
+    data instead of the flush buffer's dirty ones.  Runs outside the timed
+    events."""
+
+    def __init__(self, dev, mode: str):
+        import torch
+        self.mode = mode
+        self.w = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        self.r = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=dev) \
+            if mode == "write+read" else None
+
+    def __call__(self):
+        self.w.zero_()
+        if self.r is not None:
+            self.r.sum()
+
+    def describe(self) -> str:
+        if self.r is None:
+            return "flushed before every step: 512 MiB memset, outside the timed events"
+        return ("flushed before every step: 512 MiB memset then a 512 MiB read, outside the "
+                "timed events (no step input or output left in L2, no dirty flush lines)")
+
+
+def make_pipeline(cfg, mode, dev, weights: str):
+    """Pipeline with the workload's inputs resident on the device and its
+    expert library quantised by the library's own kernel.  ``weights``:
+    "numpy" draws them by the seeded recipe (the CPU oracle's inputs), "torch"
+    draws N(0, 0.02) with torch's CUDA generator (same distribution, seconds
+    instead of minutes for multi-GB libraries)."""
     import torch
-    import torch.distributed as dist
-
-    from permute_fp4_dispatch_b200.build import build
     from permute_fp4_dispatch_b200.pipeline import RoutingPipeline
-
-    build()
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
-    cfg = wl.config(args.config)
-    mode = cfg.modes[0]
-    x, ids, rw = wl.activations_bf16(cfg), wl.routing(cfg), wl.router_weights(cfg)
-
     pipe = RoutingPipeline(cfg.N, cfg.K, cfg.E, cfg.top_k, cfg.N_out, mode=mode,
                            epilogue=cfg.epilogue, device=dev)
-    # pinned host copies of the step's inputs (for the end-to-end measurement)
-    # a step's inputs live in one pinned host buffer laid out like the device
-    # input arena, so they travel in one copy
-    h_in, h_views = pipe.host_inputs()
-    h_x, h_ids, h_rw, h_real = (h_views[k] for k in ("x", "routing_map", "router_weights",
-                                                       "real_token_count"))
-    h_x.copy_(torch.from_numpy(x.view(np.int16)).view(torch.bfloat16))
-    h_ids.copy_(torch.from_numpy(ids))
-    h_rw.copy_(torch.from_numpy(rw))
-    h_real.fill_(cfg.real)
-    h_out = torch.empty((cfg.N, cfg.N_out), dtype=torch.bfloat16).pin_memory()
-    pipe.x.copy_(h_x)
-    pipe.routing_map.copy_(h_ids)
-    pipe.router_weights.copy_(h_rw)
-    pipe.real_token_count.copy_(h_real)
-    for e0 in range(0, cfg.E, 16):
-        es = list(range(e0, min(cfg.E, e0 + 16)))
-        pipe.quantize_weights(torch.from_numpy(wl.expert_weights_f32_many(cfg, es)).to(dev),
-                              expert_base=e0)
-        torch.cuda.synchronize()
+    h_in, views = pipe.host_inputs()
+    x, ids, rw = wl.activations_bf16(cfg), wl.routing(cfg), wl.router_weights(cfg)
+    views["x"].copy_(torch.from_numpy(x.view(np.int16)).view(torch.bfloat16))
+    views["routing_map"].copy_(torch.from_numpy(ids))
+    views["router_weights"].copy_(torch.from_numpy(rw))
+    views["real_token_count"].fill_(cfg.real)
+    pipe.inputs.copy_(h_in)
+    chunk = 16
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1000 + cfg.seed)
+    for e0 in range(0, cfg.E, chunk):
+        e1 = min(cfg.E, e0 + chunk)
+        if weights == "numpy":
+            w = torch.from_numpy(wl.expert_weights_f32_many(cfg, range(e0, e1))).to(dev)
+        else:
+            w = torch.randn((e1 - e0, cfg.N_out, cfg.K), generator=gen, device=dev) * 0.02
+        pipe.quantize_weights(w, expert_base=e0)
+        del w
+    torch.cuda.synchronize()
+    return pipe, h_in
 
+
+def measure_workload(cfg, mode, dev, steps, warmup, flush, peaks, weights, headline=False,
+                     world=1):
+    """Device-timed steps of the captured pipeline, per-kernel times, the
+    whole-step and per-kernel HBM fractions, and the end-to-end step through
+    the public API with host buffers.  Returns (record, extras)."""
+    import torch
+    pipe, h_in = make_pipeline(cfg, mode, dev, weights)
+    h_out = torch.empty((cfg.N, cfg.N_out), dtype=torch.bfloat16).pin_memory()
     stream = torch.cuda.Stream(device=dev)
     side = torch.cuda.Stream(device=dev)   # MXFP4 dispatch, concurrent with the GEMV
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    ev = lambda: torch.cuda.Event(enable_timing=True, external=True)  # noqa: E731
-    g_ev = (ev(), ev())
     with torch.cuda.stream(stream):
-        pipe.routing_map.copy_(h_ids)
-        pipe.run(stream, side_stream=side)                 # warm-up outside capture
+        pipe.run(stream, side_stream=side)               # warm-up outside capture
     stream.synchronize()
     stats = pipe.expert_usage_stats.cpu().numpy().view(np.uint32)
     A = int(stats[1])
     R = int(pipe.expert_start_indices[-1].item())
     routed_tokens = int((pipe.restore_token_order.view(cfg.N, cfg.top_k) != -1)
                         .any(dim=1).sum().item())
+    hbm_peak, bf16_peak = peaks["hbm_gbs"], peaks["bf16_tflops"]
 
     # masking is idempotent for a fixed real_token_count, so replays need no map restore
-    # The step graph as a user runs it, and the same step with two timing events
-    # around the GEMV (recorded from a side stream, so the programmatic launches
-    # stay intact).  Event-record nodes add about 3 us of graph overhead to a
-    # step, so the headline steps replay the first graph and the GEMV's launch
-    # time comes from K further timed steps of the second.
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.stream(stream):
         with torch.cuda.graph(graph, stream=stream):
             pipe.run(stream, side_stream=side)
-    graph_t = torch.cuda.CUDAGraph()
-    with torch.cuda.stream(stream):
-        with torch.cuda.graph(graph_t, stream=stream):
-            pipe.run(stream, gemv_events=g_ev, side_stream=side)
 
-    def timed_steps(n, g, gemv_times=False):
+    def replay_times(n, g, after=None):
         starts = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
         ends = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
-        gs = []
+        extra = []
         for i in range(n):
             with torch.cuda.stream(stream):
-                flush.zero_()
+                flush()
                 starts[i].record(stream)
                 g.replay()
                 ends[i].record(stream)
             ends[i].synchronize()
-            if gemv_times:
-                # gemv events are re-recorded by every replay: read them before the next one
-                gs.append(g_ev[0].elapsed_time(g_ev[1]))
+            if after is not None:
+                extra.append(after())
         torch.cuda.synchronize()
-        return [starts[i].elapsed_time(ends[i]) for i in range(n)], gs
+        return [starts[i].elapsed_time(ends[i]) for i in range(n)], extra
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    timed_steps(args.warmup, graph)
-    timed_steps(args.warmup, graph_t, True)
-    barrier()
+    replay_times(warmup, graph)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(local_rank) as clk:
-        t_step, _ = timed_steps(args.steps, graph)
-        _, t_gemv = timed_steps(args.steps, graph_t, True)
-        torch.cuda.synchronize()
-    barrier()
-    clocks = clk.summary()
+    t_step, _ = replay_times(steps, graph)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
     ms_step = max_over_ranks(float(np.mean(t_step)), world, dev)
-    ms_gemv = float(np.mean(t_gemv))
+
+    # per-kernel times: a CUDA graph of the same steps on one stream with a
+    # timing event recorded between consecutive kernels (each kernel then
+    # waits for the previous one to finish: no programmatic overlap), L2
+    # flushed before every replay
+    steps_k = pipe.kernel_steps()
+    names = [n for n, _ in steps_k]
+    kev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(names) + 1)]
+    kgraph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        for _, fn in steps_k:                            # warm-up outside capture
+            fn(stream)
+        with torch.cuda.graph(kgraph, stream=stream):
+            kev[0].record(stream)
+            for i, (_, fn) in enumerate(steps_k):
+                fn(stream)
+                kev[i + 1].record(stream)
+    _, rows = replay_times(warmup + steps, kgraph,
+                           after=lambda: [kev[i].elapsed_time(kev[i + 1]) for i in range(len(names))])
+    per = {n: [row[i] for row in rows[warmup:]] for i, n in enumerate(names)}
+    bytes_ = algorithmic_bytes(cfg, mode, A, R, routed_tokens)
+    kernels = {}
+    for n in names:
+        us = float(np.mean(per[n])) * 1e3
+        b = sum(bytes_[k] for k in KERNEL_BYTES.get(n, (n,)))
+        rec = {"us": us, "algorithmic_bytes": b, "gbs": b / (us * 1e-6) / 1e9,
+               "hbm_frac": b / (us * 1e-6) / 1e9 / hbm_peak}
+        if n == "grouped_gemv":
+            fl = dense_flops(cfg, R)
+            rec["tflops"] = fl / (us * 1e-6) / 1e12
+            rec["tensor_frac_of_bf16_peak"] = rec["tflops"] / bf16_peak
+        kernels[n] = rec
+    total_bytes = sum(bytes_.values())
 
     # end to end through the public API, host buffers: one CUDA graph per step
     # holding the H2D copy of the step's inputs from pinned memory (routing
@@ -408,12 +473,8 @@ def run_ours(args, rank, world, local_rank):
     # create_indices) and the pipeline, whose combine stores the step's result
     # straight into pinned host memory (a device-accessible pointer under
     # unified addressing), so the result crosses PCIe without a separate copy
-    e2e_ms = []
-    h2d = h_in.numel()   # routing map, router weights, real_token_count, x (+ alignment gaps)
-    d2h = h_out.numel() * 2
     xcopy = torch.cuda.Stream(device=dev)
     rb = pipe.routing_bytes
-    e2e_graph = torch.cuda.CUDAGraph()
 
     def e2e_step_ops():
         cur = torch.cuda.current_stream()
@@ -427,6 +488,7 @@ def run_ours(args, rank, world, local_rank):
         x_ready.record(xcopy)
         pipe.run(cur, side_stream=side, x_ready=x_ready)
 
+    e2e_graph = torch.cuda.CUDAGraph()
     dev_out = pipe.output
     pipe.output = h_out                                   # the combine's output buffer
     with torch.cuda.stream(stream):
@@ -435,62 +497,129 @@ def run_ours(args, rank, world, local_rank):
             e2e_step_ops()
     pipe.output = dev_out
     stream.synchronize()
-    for i in range(args.warmup + args.steps):
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            flush.zero_()
-            e0.record(stream)
-            e2e_graph.replay()
-            e1.record(stream)
-        e1.synchronize()
-        if i >= args.warmup:
-            e2e_ms.append(e0.elapsed_time(e1))
-    torch.cuda.synchronize()
+    t_e2e, _ = replay_times(warmup + steps, e2e_graph)
+    e2e_ms = max_over_ranks(float(np.mean(t_e2e[warmup:])), world, dev)
     # the result that reached the host is the device step's result
     with torch.cuda.stream(stream):
         graph.replay()
     stream.synchronize()
     assert torch.equal(h_out.view(torch.int16), pipe.output.cpu().view(torch.int16))
-    e2e_step = max_over_ranks(float(np.mean(e2e_ms)), world, dev)
 
-    peak, peak_src = measured_peaks()
-    bytes_ = algorithmic_bytes(cfg, mode, A, R, routed_tokens)
+    record = {
+        "mode": mode, "routed_pairs": R, "active_experts": A, "steps": steps,
+        "us_per_step": ms_step * 1e3, "pairs_per_s": job_rate(R, world, ms_step),
+        "kernels_us_source": ("CUDA events between consecutive kernels inside one captured "
+                              "graph of the same steps (serialised, no programmatic overlap)"),
+        "kernels": kernels,
+        "pipeline_hbm": {"algorithmic_bytes": total_bytes,
+                         "achieved_gbs": total_bytes / (ms_step * 1e-3) / 1e9,
+                         "frac": total_bytes / (ms_step * 1e-3) / 1e9 / hbm_peak},
+        "e2e": {"us_per_step": e2e_ms * 1e3, "pairs_per_s": job_rate(R, world, e2e_ms),
+                "h2d_bytes_per_step": h_in.numel(), "d2h_bytes_per_step": h_out.numel() * 2},
+        "weights": ("seeded numpy recipe" if weights == "numpy"
+                    else "N(0,0.02) from torch's CUDA generator"),
+        "gpu_launches_per_step": pipe.launches_per_run(),
+    }
+    extras = {"pipe": pipe, "graph": graph, "kgraph": kgraph, "stream": stream, "side": side,
+              "bytes": bytes_,
+              "replay_times": replay_times, "e2e_graph": e2e_graph, "A": A, "R": R,
+              "routed_tokens": routed_tokens}
+    return record, extras
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+
+    from permute_fp4_dispatch_b200.build import build
+
+    build()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    cfg = wl.config(args.config)
+    mode = cfg.modes[0]
+    peaks = measured_peaks()
+    flush = L2Flush(dev, args.flush)
+
+    with ClockSampler(local_rank) as clk:
+        head, ex = measure_workload(cfg, mode, dev, args.steps, args.warmup, flush, peaks,
+                                    weights="numpy", headline=True, world=world)
+        # the GEMV's own launch time: K further steps of the same graph with two
+        # timing events around the GEMV, recorded from a side stream so the
+        # programmatic launches stay intact (event-record nodes add graph time,
+        # so the headline steps replay the graph without them)
+        pipe, stream, side = ex["pipe"], ex["stream"], ex["side"]
+        ev = lambda: torch.cuda.Event(enable_timing=True, external=True)  # noqa: E731
+        g_ev = (ev(), ev())
+        graph_t = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            with torch.cuda.graph(graph_t, stream=stream):
+                pipe.run(stream, gemv_events=g_ev, side_stream=side)
+        ex["replay_times"](args.warmup, graph_t)
+        _, t_gemv = ex["replay_times"](args.steps, graph_t,
+                                       after=lambda: g_ev[0].elapsed_time(g_ev[1]))
+        workloads = {}
+        if world == 1 and not args.no_workloads:
+            for name in OTHER_WORKLOADS:
+                if name == cfg.name:
+                    continue
+                wc = wl.config(name)
+                recs = {}
+                for m in wc.modes:
+                    rec, wex = measure_workload(
+                        wc, m, dev, min(args.steps, WORKLOAD_STEPS_CAP), min(args.warmup, 3),
+                        flush, peaks, weights="numpy" if name == "tiny" else "torch")
+                    recs[m] = rec
+                    del wex
+                    torch.cuda.empty_cache()
+                workloads[name] = recs if len(recs) > 1 else next(iter(recs.values()))
+    clocks = clk.summary()
+
+    ms_step = head["us_per_step"] * 1e-3
+    ms_gemv = float(np.mean(t_gemv))
+    R, A = ex["R"], ex["A"]
+    bytes_ = ex["bytes"]
+    hbm = peaks["hbm_gbs"]
     gemv_gbs = bytes_["grouped_gemv"] / (ms_gemv * 1e-3) / 1e9
     total_bytes = sum(bytes_.values())
     line = {
         "metric": METRIC,
-        "value": job_rate(R, world, ms_step),
+        "value": head["pairs_per_s"],
         "unit": "routed pairs/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "fp4xbf16->f32" if mode == "w4a16" else "fp4xfp4->f32",
         "data": "synthetic (seeded; weights N(0,0.02) quantised to NVFP4 on device)",
         "config": dict(workload_config(cfg, mode, R, A),
-                       l2="flushed before every step (512 MiB memset outside the timed events)",
+                       l2=flush.describe(),
                        graph=("one CUDA graph per step: mask + create_indices, GEMV, "
                               "combine, chained by programmatic dependent launch, the "
                               "dispatch on a stream forked after mask + create_indices, "
                               "beside the GEMV; the GEMV's launch time from K more steps of "
                               "the same graph with timing events around it")),
         "roofline": {"kernel": "grouped_gemv_nvfp4", "bound": "hbm", "achieved": gemv_gbs,
-                     "peak": peak, "unit": "GB/s", "frac": gemv_gbs / peak,
+                     "peak": hbm, "unit": "GB/s", "frac": gemv_gbs / hbm,
                      "traffic": profiled_traffic(cfg.name),
                      "algorithmic_bytes": bytes_["grouped_gemv"], "us_per_launch": ms_gemv * 1e3,
-                     "peak_source": peak_src},
+                     "peak_source": peaks["source"]},
         "pipeline_roofline": {"algorithmic_bytes": total_bytes,
                               "achieved_gbs": total_bytes / (ms_step * 1e-3) / 1e9,
-                              "frac": total_bytes / (ms_step * 1e-3) / 1e9 / peak,
+                              "frac": total_bytes / (ms_step * 1e-3) / 1e9 / hbm,
                               "bytes_by_kernel": bytes_},
-        "e2e": {"value": job_rate(R, world, e2e_step), "unit": "routed pairs/s",
-                "ms_per_step": e2e_step, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "kernels": head["kernels"],
+        "e2e": {"value": head["e2e"]["pairs_per_s"], "unit": "routed pairs/s",
+                "ms_per_step": head["e2e"]["us_per_step"] * 1e-3,
+                "h2d_bytes_per_step": head["e2e"]["h2d_bytes_per_step"],
+                "d2h_bytes_per_step": head["e2e"]["d2h_bytes_per_step"]},
         "gpu_launches": pipe.launches_per_run() * args.steps,
         "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
     }
+    if workloads:
+        line["workloads"] = workloads
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg, mode, args.cpu_sample_tokens)
     if rank == 0:
         print(json.dumps(line), flush=True)
-    del graph, graph_t, e2e_graph
+    del graph_t, ex
 
 
 def main():

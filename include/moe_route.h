@@ -160,7 +160,10 @@ MOE_API moe_status_t moe_mask_and_create_indices(int64_t *routing_map, int32_t N
 /*     must be serialised by the caller.                                 */
 /*   - The first call on each device looks up the array's device address */
 /*     (cudaGetSymbolAddress, with that device current); make that first */
-/*     call before starting any stream capture.                          */
+/*     call before starting any stream capture.  The address is cached   */
+/*     per device for the life of the process: do not use this entry     */
+/*     point after cudaDeviceReset, nor from a context other than the    */
+/*     device's primary context (the cached address belongs to it).      */
 #define MOE_CREATE_INDICES_STATIC_SCRATCH ((size_t)262144)
 MOE_API moe_status_t moe_create_indices_static(const int64_t *topk_ids, int64_t num_slots,
                                                int32_t E, uint32_t *token_expert_order,
@@ -220,33 +223,47 @@ MOE_API moe_status_t moe_quantize_weights_nvfp4(const float *w, int32_t E, int32
 
 /* --------------------------------------------------------------------- */
 /* Step 4b -- FlashRT "grouped-moe-gemv" card: grouped_w4a16_gemv_bf16 /  */
-/* grouped_w4a4_gemv_bf16 (token-major routing: activations [M, K],      */
-/* indices [M, top_k], library [E, N, K/2], output [M, top_k, N]).        */
-/* For every routed pair p = m*top_k + j with expert e:                  */
+/* grouped_w4a4_gemv_bf16, token-major routing (W4A4 routing paragraph:  */
+/* activations [M, K], device indices [M, top_k], library [E, N, K/2],    */
+/* output [M, top_k, N]).  For every routed pair p = m*top_k + j with     */
+/* expert e = indices[m, j] in [0, E):                                   */
 /*   out[p, n] = bf16( g_w[e] * g_a * sum_k a(m,k) * w(e,n,k) )           */
 /* accumulated in fp32, where w = e2m1(wq) * e4m3(sfw) and               */
 /*   MOE_W4A16: a = act (bf16 [M, K]), sfa = NULL, g_a = act_global;     */
 /*   MOE_W4A4 : a = e2m1(act) * e4m3(sfa), act uint8 [M, K/2],           */
 /*              sfa uint8 [M, K/16] (from step 4a), g_a = act_global.    */
-/* Unrouted slots of out are not written.  The pairs and their experts   */
-/* are read from the moe_create_indices outputs for the same routing map */
-/* (token_expert_order, expert_start_indices, expert_ids,                */
-/* expert_usage_stats), so "M = routed pairs, top_k = 1" is simply a     */
-/* routing map of shape [R, 1].  w_global may be NULL (all ones).        */
-/* Limits: K % 64 == 0, N % 8 == 0, 1 <= top_k <= E <= 1024; act, w and */
-/* out 16-byte aligned.  W4A16 activations enter the tensor cores as     */
-/* fp16: exact for 2^-14 <= |x| <= 65504, rounded to fp16 subnormals     */
-/* below (absolute error <= 2^-25); |x| > 65504 raises                   */
-/* MOE_DEVERR_ACT_RANGE (the affected outputs are then undefined).       */
+/* Slots whose id is outside [0, E) are not written.                     */
+/*   indices   int64 [M, top_k], device memory (its values may change     */
+/*             between CUDA-graph replays)                                */
+/*   w_global  fp32 [E] or NULL (all ones)                                */
+/*   grouping  token_expert_order, expert_start_indices, expert_ids,      */
+/*             expert_usage_stats: EITHER all four, the moe_create_indices */
+/*             outputs for this same map (then indices may be NULL), OR   */
+/*             all four NULL: the call then groups the pairs of indices   */
+/*             itself (one extra launch) into `workspace`, which must hold */
+/*             moe_grouped_gemv_workspace_bytes(M, top_k, E) bytes, 256-  */
+/*             byte aligned, caller-owned, contents need no initialisation */
+/*             (with the grouping given, workspace may be NULL)           */
+/* "M = routed pairs, top_k = 1" is simply a routing map of shape [R, 1]. */
+/* Limits: K % 32 == 0, N % 8 == 0, 1 <= top_k <= E <= 1024; act, w, sfw  */
+/* and out 16-byte aligned, sfa 4-byte aligned.  W4A4 with K % 64 == 0 runs */
+/* on the block-scaled FP4 tensor core (both operands stay NVFP4).  Errors: MOE_ERR_INVALID_ARG (shapes, nulls,  */
+/* alignment, a partial grouping), MOE_ERR_WORKSPACE (missing or small    */
+/* workspace when the grouping is not given); nothing is launched then.   */
+/* W4A16 activations enter the tensor cores as fp16: exact for            */
+/* 2^-14 <= |x| <= 65504, rounded to fp16 subnormals below (absolute      */
+/* error <= 2^-25); |x| > 65504 raises MOE_DEVERR_ACT_RANGE (the affected  */
+/* outputs are then undefined).                                           */
+MOE_API size_t moe_grouped_gemv_workspace_bytes(int32_t M, int32_t top_k, int32_t E);
 MOE_API moe_status_t moe_grouped_gemv_nvfp4(moe_gemv_mode_t mode, const void *act, const uint8_t *sfa,
-                                    float act_global, int32_t M, int32_t top_k,
-                                    const uint8_t *w, const uint8_t *sfw, const float *w_global,
-                                    int32_t E, int32_t N, int32_t K,
+                                    float act_global, const int64_t *indices, int32_t M,
+                                    int32_t top_k, const uint8_t *w, const uint8_t *sfw,
+                                    const float *w_global, int32_t E, int32_t N, int32_t K,
                                     const uint32_t *token_expert_order,
                                     const uint32_t *expert_start_indices,
                                     const int32_t *expert_ids,
                                     const uint32_t *expert_usage_stats, void *out,
-                                    cudaStream_t s);
+                                    void *workspace, size_t ws_bytes, cudaStream_t s);
 
 /* --------------------------------------------------------------------- */
 /* Step 5 -- MAX "Struct_ep_combine_wait", execute() (weighted sum with  */

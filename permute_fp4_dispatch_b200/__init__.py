@@ -25,7 +25,8 @@ __all__ = [
     "moe_create_indices_static", "MOE_CREATE_INDICES_STATIC_SCRATCH",
     "moe_mask_and_create_indices",
     "moe_mxfp4_row_stride", "moe_dispatch_mxfp4", "moe_quantize_activations_nvfp4",
-    "moe_quantize_weights_nvfp4", "moe_grouped_gemv_nvfp4", "moe_combine",
+    "moe_quantize_weights_nvfp4", "moe_grouped_gemv_workspace_bytes", "moe_grouped_gemv_nvfp4",
+    "moe_combine",
     "moe_status_string", "moe_get_device_error", "moe_version",
 ]
 
@@ -59,8 +60,9 @@ _SIGS = {
     "moe_dispatch_mxfp4": ([_P, _I32, _I32, _I32, _I32, _P, _P, _P, _P, _P, _I64, _P, _P], _I32),
     "moe_quantize_activations_nvfp4": ([_P, _I32, _I32, _F32, _P, _P, _P], _I32),
     "moe_quantize_weights_nvfp4": ([_P, _I32, _I32, _I32, _P, _P, _P, _P], _I32),
-    "moe_grouped_gemv_nvfp4": ([_I32, _P, _P, _F32, _I32, _I32, _P, _P, _P, _I32, _I32, _I32,
-                                _P, _P, _P, _P, _P, _P], _I32),
+    "moe_grouped_gemv_workspace_bytes": ([_I32, _I32, _I32], _SZ),
+    "moe_grouped_gemv_nvfp4": ([_I32, _P, _P, _F32, _P, _I32, _I32, _P, _P, _P, _I32, _I32, _I32,
+                                _P, _P, _P, _P, _P, _P, _SZ, _P], _I32),
     "moe_combine": ([_P, _P, _P, _I32, _I32, _I32, _I32, _I32, _F32, _P, _P], _I32),
     "moe_status_string": ([_I32], ctypes.c_char_p),
     "moe_get_device_error": ([_P, _I32], _I32),
@@ -189,14 +191,22 @@ def moe_quantize_weights_nvfp4(w, E: int, N: int, K: int, wq, sfw, w_global, str
         "moe_quantize_weights_nvfp4")
 
 
-def moe_grouped_gemv_nvfp4(mode: int, act, sfa, act_global: float, M: int, top_k: int, w, sfw,
-                           w_global, E: int, N: int, K: int, token_expert_order,
-                           expert_start_indices, expert_ids, expert_usage_stats, out,
-                           stream=None):
+def moe_grouped_gemv_workspace_bytes(M: int, top_k: int, E: int) -> int:
+    return library().moe_grouped_gemv_workspace_bytes(M, top_k, E)
+
+
+def moe_grouped_gemv_nvfp4(mode: int, act, sfa, act_global: float, indices, M: int, top_k: int,
+                           w, sfw, w_global, E: int, N: int, K: int, token_expert_order=None,
+                           expert_start_indices=None, expert_ids=None, expert_usage_stats=None,
+                           out=None, workspace=None, ws_bytes: int = 0, stream=None):
+    """Grouped GEMV over the routing map ``indices`` [M, top_k].  Pass the
+    four moe_create_indices outputs for this map, or none of them and a
+    workspace of moe_grouped_gemv_workspace_bytes(M, top_k, E) bytes."""
     _check(library().moe_grouped_gemv_nvfp4(
-        mode, _ptr(act), _ptr(sfa), act_global, M, top_k, _ptr(w), _ptr(sfw), _ptr(w_global),
-        E, N, K, _ptr(token_expert_order), _ptr(expert_start_indices), _ptr(expert_ids),
-        _ptr(expert_usage_stats), _ptr(out), _stream(stream)), "moe_grouped_gemv_nvfp4")
+        mode, _ptr(act), _ptr(sfa), act_global, _ptr(indices), M, top_k, _ptr(w), _ptr(sfw),
+        _ptr(w_global), E, N, K, _ptr(token_expert_order), _ptr(expert_start_indices),
+        _ptr(expert_ids), _ptr(expert_usage_stats), _ptr(out), _ptr(workspace), ws_bytes,
+        _stream(stream)), "moe_grouped_gemv_nvfp4")
 
 
 def moe_combine(expert_out, router_weights, topk_ids, M: int, top_k: int, H: int, E: int,

@@ -6,11 +6,11 @@
 // are already local, so there is no wait phase.
 //
 // One warp per (token, 256-column segment): each lane owns 8 columns.  The
-// rows of the first eight slots are requested at once, together with the
-// token's slot ids and weights (one slot per lane); the routed ones among
-// them, then the routed slots beyond eight (128-bit loads, up to eight in
-// flight), are accumulated in fp32 in slot order and written as 8 bf16 with
-// one 128-bit store.  Rows of unrouted slots are never used.
+// token's slot ids and weights are read first (one slot per lane); then only
+// the routed slots' rows are loaded (128-bit loads, up to eight in flight),
+// accumulated in fp32 in slot order and written as 8 bf16 with one 128-bit
+// store.  Rows of unrouted slots -- which the GEMV never wrote -- are never
+// read, so padding rows of a CUDA-graph bucket cost their metadata only.
 #pragma once
 #include "common.cuh"
 
@@ -35,14 +35,6 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
     const int h = (int)(w % segs) * 256 + 8 * (int)lane;
     const bool col_ok = h < H;
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    // the first (up to) 8 slots' rows are requested together with the slot
-    // metadata; rows of unrouted slots arrive but are not used
-    constexpr int kEarly = 8;
-    uint4 ve[kEarly];
-#pragma unroll
-    for (int b = 0; b < kEarly; ++b)
-      ve[b] = (b < top_k && col_ok) ? ldg_nc_v4(y + ((t * top_k + b) * H + h))
-                                    : make_uint4(0u, 0u, 0u, 0u);
     for (int j0 = 0; j0 < top_k; j0 += 32) {
       const int jl = j0 + (int)lane;
       bool ok = false;
@@ -53,25 +45,6 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32)
         wl = rw[t * top_k + jl];
       }
       unsigned m = __ballot_sync(0xffffffffu, ok);
-      if (j0 == 0) {
-        // slots below kEarly: rows already loaded, accumulated in slot order
-        const unsigned early = m & ((1u << kEarly) - 1u);
-#pragma unroll
-        for (int b = 0; b < kEarly; ++b) {
-          if (early & (1u << b)) {
-            const float wt = __shfl_sync(0xffffffffu, wl, b);
-            acc[0] = fmaf(wt, bf16_lo(ve[b].x), acc[0]);
-            acc[1] = fmaf(wt, bf16_hi(ve[b].x), acc[1]);
-            acc[2] = fmaf(wt, bf16_lo(ve[b].y), acc[2]);
-            acc[3] = fmaf(wt, bf16_hi(ve[b].y), acc[3]);
-            acc[4] = fmaf(wt, bf16_lo(ve[b].z), acc[4]);
-            acc[5] = fmaf(wt, bf16_hi(ve[b].z), acc[5]);
-            acc[6] = fmaf(wt, bf16_lo(ve[b].w), acc[6]);
-            acc[7] = fmaf(wt, bf16_hi(ve[b].w), acc[7]);
-          }
-        }
-        m &= ~((1u << kEarly) - 1u);
-      }
       while (m) {
         // a batch of up to 8 routed slots: issue all loads, then accumulate in order
         uint4 v[8];

@@ -174,10 +174,30 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of a phase's completion.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait: returns false (and raises MOE_DEVERR_WAIT_TIMEOUT) when the
-// phase has not completed within `limit_ns` nanoseconds.
+// phase has not completed within `limit_ns` nanoseconds.  A limit of 0 means
+// "no waiting at all": only a phase that has already completed passes (a
+// try_wait may suspend the thread for a while, so it is not used then).
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity,
                                                   uint64_t limit_ns) {
+  if (limit_ns == 0) {
+    if (mbar_test_wait(bar, parity)) return true;
+    raise_device_error(MOE_DEVERR_WAIT_TIMEOUT);
+    return false;
+  }
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
@@ -378,5 +398,55 @@ __device__ __forceinline__ void umma_commit(uint64_t *bar) {
       "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
           smem_addr(bar))
       : "memory");
+}
+}  // namespace moe
+
+namespace moe {
+// ------------------------------------------------------------------ block-scaled FP4 tensor core
+// Instruction descriptor, kind::mxf4nvf4 with E4M3 scales per 16 elements:
+// A and B E2M1 (K-major), fp32 D, M x N, K = 64 per instruction; both
+// scale-factor byte selectors 0 (all four bytes of a TMEM word are used).
+__host__ __device__ constexpr uint32_t umma_idesc_nvf4(int M, int N) {
+  return (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+// D[tmem] (+)= (A[smem] x SFA[tmem]) * (B[smem] x SFB[tmem])^T, issued by one thread.
+__device__ __forceinline__ void umma_nvf4_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                             uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], "
+      "p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+// Shared-memory descriptor of a K-major block without swizzle whose rows are
+// 16 bytes apart, 8-row groups `sbo` bytes apart (source of tcgen05.cp).
+__device__ __forceinline__ uint64_t smem_desc_interleave(uint32_t saddr, uint32_t sbo) {
+  uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)1u << 16;                          // leading byte offset (16 B, unused)
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;      // stride byte offset
+  d |= (uint64_t)1u << 46;                          // descriptor version (sm_100)
+  return d;                                         // layout type 0: no swizzle
+}
+// Copy 32 rows x 16 bytes from shared memory into TMEM lanes 0-31, columns
+// [col, col + 4), replicated into the other three lane quadrants.
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+               : "memory");
+}
+// cp.async of `bytes` (4 or 16) with zero fill of the part beyond `src_bytes`.
+__device__ __forceinline__ void cp_async4_zfill(void *dst, const void *src, uint32_t src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_addr(dst)), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async16_zfill(void *dst, const void *src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_addr(dst)), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
 }
 }  // namespace moe

@@ -1,0 +1,342 @@
+// gemv_bs.cuh -- step 4b, W4A4 on the block-scaled FP4 tensor core.
+//
+// FlashRT "grouped-moe-gemv" card (Available functions: grouped_w4a4_gemv_bf16;
+// hardware list: block-scaled-MMA W4A4).  For each routed pair p with expert e:
+//     out[p, n] = bf16( g_w[e] * g_a * sum_k e2m1(xq[m,k]) e4m3(sfa[m,k/16])
+//                                       * e2m1(wq[e,n,k]) e4m3(sfw[e,n,k/16]) ).
+// Both operands stay in their NVFP4 encoding all the way into the tensor
+// core: tcgen05.mma.kind::mxf4nvf4.block_scale with 16-element E4M3 scale
+// vectors multiplies the raw E2M1 codes and applies both scale factors, so
+// nothing is dequantised on the CUDA cores.
+//
+// Design (one persistent CTA per SM, 6 warps):
+//   * Work units are (active expert a, 128-row block rb, pass p of up to
+//     kTS = 128 tokens), in that order, so the passes of one row block follow
+//     each other and a block's weights are read from HBM once even when its
+//     expert holds more tokens than one pass.  The CTAs take equal contiguous
+//     ranges of units.  One unit is one MMA tile: M = 128 weight rows (A),
+//     N = the pass's tokens rounded up to 16 (B), fp32 D in tensor memory.
+//   * warp 0, lane 0: streams the unit's weight codes, 128 rows x 256 codes
+//     per stage, with one TMA box (128B swizzle, L2 evict-first; rows past N
+//     and codes past K arrive as zeros) into a kStages-deep ring;
+//   * warps 2-5 (128 threads): per stage, gather the pass's token rows
+//     (128 bytes of codes each) into the 128B-swizzled K-major B tile, and
+//     the stage's scale factors of both operands into shared memory in the
+//     tensor core's 32-row x 16-byte scale layout, all with cp.async (zero
+//     fill past K, past N and past the pass's tokens), arriving on the
+//     stage's barrier when the copies land; they also run the epilogue
+//     (tensor memory -> scale by g_w * g_a -> bf16 -> out) of the previous
+//     unit while the next one streams;
+//   * warp 1, lane 0: owns tensor memory; per stage copies the scale
+//     factors into it (tcgen05.cp 32x128b, replicated over the four lane
+//     quadrants) and issues four kind::mxf4nvf4 MMAs of K = 64, committing
+//     to the barrier that frees the stage; D is double-buffered, so a unit's
+//     epilogue overlaps the next unit's MMAs.
+//   * Every wait is bounded; an expired wait raises MOE_DEVERR_WAIT_TIMEOUT,
+//     the roles stop issuing, wait (bounded) for their copies and MMAs in
+//     flight, and the CTA releases tensor memory and returns.
+#pragma once
+#include "gemv_common.cuh"
+
+namespace moe {
+namespace gemv {
+namespace bs {
+
+constexpr int kProdWarp = 0;
+constexpr int kMmaWarp = 1;
+constexpr int kSW0 = 2;                   // first staging / epilogue warp
+constexpr int kSWThreads = 4 * 32;
+constexpr int kThreads = 2 * 32 + kSWThreads;
+constexpr int kKC = 256;                  // codes per stage: 128 bytes of each row
+constexpr int kKSteps = kKC / 64;         // MMAs (K = 64) per stage
+constexpr int kTS = 128;                  // tokens per pass
+constexpr int kStages = 5;
+constexpr int kATile = 128 * 128;         // weight tile: 128 rows x 128 bytes
+constexpr int kBTile = kTS * 128;         // token tile: 128 rows x 128 bytes
+constexpr int kSFStep = 512;              // one operand's scales for one MMA: 32 rows x 16 B
+constexpr int kSFBytes = kKSteps * kSFStep;
+constexpr int kStageBytes = kATile + kBTile + 2 * kSFBytes;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kDcol = 0;             // D: two buffers of kTS columns
+constexpr uint32_t kSFcol = 2 * kTS;      // per stage: 16 columns of A scales, 16 of B scales
+static_assert(kSFcol + kStages * 32 <= kTmemCols, "tensor memory columns");
+static_assert(kStageBytes % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
+
+constexpr size_t kOffStart = (size_t)kStages * kStageBytes;
+constexpr size_t kOffEid = kOffStart + (kMaxExperts + 4) * 4;
+constexpr size_t kOffPrefix = kOffEid + (kMaxExperts + 4) * 4;
+constexpr size_t kOffPair = kOffPrefix + (kMaxExperts + 4) * 4;  // [2][kTS] pair ids
+constexpr size_t kOffBar = kOffPair + 2 * kTS * 4;
+constexpr int kNumBars = 3 * kStages + 5;
+constexpr size_t kOffMisc = kOffBar + kNumBars * 8;              // tmem slot, abort flag
+constexpr size_t kSmemBytes = kOffMisc + 16 + 1024;              // + alignment slack
+static_assert(kSmemBytes <= 232448, "shared memory per block");
+
+struct Unit {
+  int e;          // expert id
+  uint32_t tok0;  // first position of the pass in token_expert_order
+  int ntok;       // tokens of the pass
+  int n0;         // first weight row of the block
+};
+
+// Walks a CTA's unit range in order; unit u of active expert a with c pairs
+// (P = ceil(c / kTS) passes) is block v / P, pass v % P, v = u - prefix[a].
+struct UnitWalk {
+  uint32_t u, u_end;
+  int a;
+  __device__ __forceinline__ bool next(const uint32_t *prefix, const uint32_t *start,
+                                       const int32_t *eid, Unit &r) {
+    if (u >= u_end) return false;
+    while (u >= prefix[a + 1]) ++a;
+    const uint32_t v = u - prefix[a];
+    const uint32_t c = start[a + 1] - start[a];
+    const uint32_t P = (c + kTS - 1) / kTS;
+    const uint32_t pass = v % P;
+    r.e = eid[a];
+    r.tok0 = start[a] + pass * kTS;
+    r.ntok = (int)min((uint32_t)kTS, c - pass * kTS);
+    r.n0 = (int)(v / P) * 128;
+    ++u;
+    return true;
+  }
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_gemv_bs_kernel(const Params p, const __grid_constant__ CUtensorMap tmap_w) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint32_t *s_start = reinterpret_cast<uint32_t *>(smem + kOffStart);
+  int32_t *s_eid = reinterpret_cast<int32_t *>(smem + kOffEid);
+  uint32_t *prefix = reinterpret_cast<uint32_t *>(smem + kOffPrefix);
+  uint32_t *s_pair = reinterpret_cast<uint32_t *>(smem + kOffPair);
+  uint64_t *a_full = reinterpret_cast<uint64_t *>(smem + kOffBar);  // weight tile landed
+  uint64_t *b_full = a_full + kStages;   // token tile and scales landed
+  uint64_t *empty = b_full + kStages;    // the stage's MMAs are done
+  uint64_t *d_full = empty + kStages;    // [2] a unit's D is complete
+  uint64_t *d_empty = d_full + 2;        // [2] a unit's D has been read out
+  uint64_t *mma_drain = d_empty + 2;     // completes once every MMA issued so far is done
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffMisc);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffMisc + 8);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = (int)lane_id();
+  // set-up that reads no input runs before the wait for the previous grid
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&a_full[s], 1u);
+      mbar_init(&b_full[s], (uint32_t)kSWThreads);
+      mbar_init(&empty[s], 1u);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&d_full[b], 1u);
+      mbar_init(&d_empty[b], 4u);
+    }
+    mbar_init(mma_drain, 1u);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kProdWarp && lane == 0) prefetch_tmap(&tmap_w);
+  if (warp == kMmaWarp) tmem_alloc(tmem_slot, kTmemCols);
+  pdl_wait();
+  pdl_launch_dependents();
+
+  const int N = p.N, K = p.K;
+  const int RB = (N + 127) / 128;
+  const uint32_t A = p.stats[1];
+  for (uint32_t i = threadIdx.x; i <= A; i += blockDim.x) {
+    s_start[i] = p.start[i];
+    if (i < A) s_eid[i] = p.eids[i];
+  }
+  __syncthreads();
+  if (warp == 0) build_prefix(prefix, s_start, A, (uint32_t)kTS, RB, lane);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+  const uint32_t U = prefix[A];
+  const uint32_t u0 = muldiv(U, blockIdx.x, gridDim.x);
+  const uint32_t u1 = muldiv(U, blockIdx.x + 1, gridDim.x);
+  const int nst = (K + kKC - 1) / kKC;
+  const int a0 = u0 < u1 ? expert_of_unit(prefix, A, u0) : 0;
+
+  auto wait = [&](uint64_t *bar, uint32_t parity) {
+    if (*abort_flag) return;
+    if (!mbar_wait_bounded(bar, parity, p.wait_limit_ns)) *abort_flag = 1;
+  };
+  auto stage = [&](int s) { return smem + (size_t)s * kStageBytes; };
+
+  if (warp == kProdWarp) {
+    // ================================================================ weight tiles (TMA)
+    if (lane == 0) {
+      const uint64_t policy = l2_evict_first_policy();
+      UnitWalk walk{u0, u1, a0};
+      Unit r;
+      uint32_t it = 0, issued = 0;
+      while (!*abort_flag && walk.next(prefix, s_start, s_eid, r)) {
+        for (int c = 0; c < nst; ++c, ++it) {
+          const int s = (int)(it % kStages);
+          wait(&empty[s], ((it / kStages) & 1u) ^ 1u);
+          if (*abort_flag) break;
+          mbar_arrive_expect_tx(&a_full[s], (uint32_t)kATile);
+          tma_load_3d(stage(s), &tmap_w, c * (kKC / 2), r.n0, r.e, &a_full[s], policy);
+          issued = it + 1;
+        }
+      }
+      // after an abort, let the copies still in flight land (bounded)
+      if (*abort_flag) {
+        for (int s = 0; s < kStages; ++s) {
+          const uint32_t fills =
+              issued > (uint32_t)s ? (issued - (uint32_t)s + kStages - 1) / kStages : 0u;
+          if (fills) mbar_wait_bounded(&a_full[s], (fills - 1) & 1u, kDrainLimitNs);
+        }
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    // ================================================================ MMA issuer
+    if (lane == 0) {
+      UnitWalk walk{u0, u1, a0};
+      Unit r;
+      uint32_t it = 0, rnd = 0;
+      while (walk.next(prefix, s_start, s_eid, r)) {
+        const uint32_t d = rnd & 1u;
+        wait(&d_empty[d], ((rnd >> 1) & 1u) ^ 1u);
+        tc_fence_after();
+        const uint32_t idesc = umma_idesc_nvf4(128, (r.ntok + 15) & ~15);
+        const uint32_t d_t = tbase + kDcol + d * (uint32_t)kTS;
+        for (int c = 0; c < nst; ++c, ++it) {
+          const int s = (int)(it % kStages);
+          wait(&a_full[s], (it / kStages) & 1u);
+          wait(&b_full[s], (it / kStages) & 1u);
+          fence_proxy_async_smem();  // token tile and scales were written by cp.async
+          tc_fence_after();
+          if (!*abort_flag) {
+            const uint8_t *st = stage(s);
+            const uint32_t a_addr = smem_addr(st), b_addr = a_addr + kATile;
+            const uint32_t sfa_addr = b_addr + kBTile, sfb_addr = sfa_addr + kSFBytes;
+            const uint32_t sf_t = tbase + kSFcol + (uint32_t)s * 32u;
+            const int ksteps = min(kKSteps, (K - c * kKC) / 64);
+            for (int kk = 0; kk < ksteps; ++kk) {
+              tmem_cp_32x128b_x4(sf_t + 4u * kk, smem_desc_interleave(sfa_addr + kk * kSFStep, 128));
+              tmem_cp_32x128b_x4(sf_t + 16u + 4u * kk,
+                                 smem_desc_interleave(sfb_addr + kk * kSFStep, 128));
+            }
+            for (int kk = 0; kk < ksteps; ++kk)
+              umma_nvf4_ss(d_t, umma_desc_sw128(a_addr + 32u * kk, 1024u),
+                           umma_desc_sw128(b_addr + 32u * kk, 1024u), idesc, sf_t + 4u * kk,
+                           sf_t + 16u + 4u * kk, (c > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(&empty[s]);
+        }
+        umma_commit(&d_full[d]);
+        ++rnd;
+      }
+      // no MMA or scale copy may still use shared or tensor memory when the CTA releases them
+      umma_commit(mma_drain);
+      mbar_wait_bounded(mma_drain, 0u, kDrainLimitNs);
+    }
+    __syncwarp();
+  } else {
+    // ================================================================ token tiles, scales, epilogue
+    const int t = (int)threadIdx.x - kSW0 * 32;  // 0 .. 127
+    const int q = warp & 3;                       // the TMEM lane quadrant this warp may access
+    const int i32 = t & 31, cq = t >> 5;          // scale row i32 + 32 * cq of the stage layout
+    const int64_t xrow = K / 2, sfrow = K / 16;
+    const uint8_t *xq = static_cast<const uint8_t *>(p.act);
+    UnitWalk walk{u0, u1, a0};
+    Unit r, rp;
+    bool have = walk.next(prefix, s_start, s_eid, r), pending = false;
+    uint32_t it = 0, rnd = 0, rnd_p = 0;
+
+    auto epilogue = [&](const Unit &er, uint32_t ernd) {
+      const uint32_t d = ernd & 1u;
+      wait(&d_full[d], (ernd >> 1) & 1u);
+      tc_fence_after();
+      const int n = er.n0 + 32 * q + lane;
+      const bool ok = !*abort_flag && n < N;
+      const float f = __fmul_rn(p.w_global ? __ldg(p.w_global + er.e) : 1.0f, p.g_a);
+      const uint32_t *pairs = s_pair + (ernd & 1u) * kTS;
+      for (int c0 = 0; c0 < er.ntok; c0 += 16) {
+        uint32_t v[16];
+        tmem_ld16(tbase + ((uint32_t)(32 * q) << 16) + kDcol + d * (uint32_t)kTS + (uint32_t)c0, v);
+        tmem_wait_ld();
+        if (ok) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            if (c0 + j < er.ntok) {
+              const __nv_bfloat16 o = __float2bfloat16_rn(__uint_as_float(v[j]) * f);
+              p.out[(int64_t)pairs[c0 + j] * N + n] = __bfloat16_as_ushort(o);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&d_empty[d]);
+    };
+
+    while (have) {
+      named_bar_sync(1, kSWThreads);  // earlier readers of this pair buffer are done
+      uint32_t *pairs = s_pair + (rnd & 1u) * kTS;
+      if (t < r.ntok) pairs[t] = __ldg(p.order + r.tok0 + t);
+      named_bar_sync(1, kSWThreads);
+      // this thread's token row of the B tile, and the rows of its scale words
+      const bool tok_ok = t < r.ntok;
+      const uint8_t *xrow_t = xq + (tok_ok ? (int64_t)(pairs[t] / (uint32_t)p.top_k) * xrow : 0);
+      const int wrow = r.n0 + i32 + 32 * cq;
+      const bool wrow_ok = wrow < N;
+      const uint8_t *sfa_src = p.sfw + ((int64_t)r.e * N + (wrow_ok ? wrow : 0)) * sfrow;
+      const bool tokb_ok = i32 + 32 * cq < r.ntok;
+      const uint8_t *sfb_src =
+          p.sfa + (tokb_ok ? (int64_t)(pairs[i32 + 32 * cq] / (uint32_t)p.top_k) * sfrow : 0);
+      for (int c = 0; c < nst; ++c, ++it) {
+        const int s = (int)(it % kStages);
+        wait(&empty[s], ((it / kStages) & 1u) ^ 1u);
+        if (!*abort_flag) {
+          uint8_t *bt = stage(s) + kATile;
+          uint8_t *sfa_s = bt + kBTile, *sfb_s = sfa_s + kSFBytes;
+          const int kb0 = c * (kKC / 2);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const bool ok = tok_ok && kb0 + 16 * (j + 1) <= xrow;
+            cp_async16_zfill(bt + t * 128 + ((j ^ (t & 7)) << 4), ok ? xrow_t + kb0 + 16 * j : xq,
+                             ok ? 16u : 0u);
+          }
+#pragma unroll
+          for (int kk = 0; kk < kKSteps; ++kk) {
+            const int kc = c * (kKC / 16) + 4 * kk;  // first scale byte of the MMA's K range
+            const bool kin = kc + 4 <= sfrow;
+            uint8_t *dst = sfa_s + kk * kSFStep + i32 * 16 + cq * 4;
+            cp_async4_zfill(dst, kin && wrow_ok ? sfa_src + kc : p.sfw, kin && wrow_ok ? 4u : 0u);
+            dst = sfb_s + kk * kSFStep + i32 * 16 + cq * 4;
+            cp_async4_zfill(dst, kin && tokb_ok ? sfb_src + kc : p.sfa, kin && tokb_ok ? 4u : 0u);
+          }
+        }
+        cp_async_mbar_arrive_noinc(&b_full[s]);
+        // the previous unit's epilogue overlaps this unit's first stage
+        if (c == 0 && pending) {
+          epilogue(rp, rnd_p);
+          pending = false;
+        }
+      }
+      rp = r;
+      rnd_p = rnd;
+      pending = true;
+      ++rnd;
+      have = walk.next(prefix, s_start, s_eid, r);
+    }
+    if (pending) epilogue(rp, rnd_p);
+    cp_async_wait_all();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tbase, kTmemCols);
+  }
+}
+
+}  // namespace bs
+}  // namespace gemv
+}  // namespace moe

@@ -10,7 +10,8 @@ namespace gemv {
 constexpr int kMaxExperts = 1024;
 constexpr int kBlocksPerRound = 8;      // 16-row blocks per round (128 rows), unless a
                                         // kernel asks for another round size
-constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: default limit of every pipeline wait
+constexpr uint64_t kDrainLimitNs = 100000000ull;  // 100 ms: waits for copies in flight after an abort
 
 struct Params {
   const void *act;          // W4A16: bf16 [M, K]; W4A4: u8 [M, K/2]
@@ -26,6 +27,7 @@ struct Params {
   const int32_t *eids;
   const uint32_t *stats;
   uint16_t *out;            // bf16 [M, top_k, N]
+  uint64_t wait_limit_ns;   // limit of each pipeline wait (kWaitLimitNs unless a test shortens it)
 };
 
 struct Round {
@@ -58,6 +60,11 @@ __device__ __forceinline__ int expert_of_unit(const uint32_t *prefix, uint32_t A
 }
 
 // Walks a CTA's unit range round by round; identical in every thread.
+// Within an active expert with c pairs (P = ceil(c / ts) passes) the units
+// (16-row blocks) are ordered by 128-row round, then pass, then block: the
+// passes over one round of weight rows follow each other, so an expert with
+// more tokens than one pass reads each round's weights from HBM once and
+// from L2 for the other passes.  A round is cut short at the range's end.
 struct RoundIter {
   uint32_t u, u_end;
   int a;
@@ -67,17 +74,28 @@ struct RoundIter {
     if (u >= u_end) return false;
     while (u >= m.prefix[a + 1]) ++a;
     const uint32_t v = u - m.prefix[a];
-    const uint32_t pass = v / (uint32_t)RB;
-    const uint32_t rb = v % (uint32_t)RB;
-    uint32_t nblk = (uint32_t)RB - rb;
-    if (nblk > round_blocks) nblk = round_blocks;
-    if (nblk > u_end - u) nblk = u_end - u;
     const uint32_t s0 = m.start[a];
     const uint32_t c = m.start[a + 1] - s0;
+    const uint32_t P = (c + ts - 1) / ts;
+    const uint32_t R8 = ((uint32_t)RB + round_blocks - 1) / round_blocks;
+    const uint32_t full = (R8 - 1) * round_blocks * P;  // units of the rounds before the last
+    uint32_t ri, rem, nb;
+    if (v < full) {
+      ri = v / (round_blocks * P);
+      rem = v - ri * round_blocks * P;
+      nb = round_blocks;
+    } else {
+      ri = R8 - 1;
+      rem = v - full;
+      nb = (uint32_t)RB - ri * round_blocks;
+    }
+    const uint32_t pass = rem / nb, bi = rem % nb;
+    uint32_t nblk = nb - bi;
+    if (nblk > u_end - u) nblk = u_end - u;
     r.e = m.eid[a];
     r.tok0 = s0 + pass * ts;
     r.ntok = (int)min(ts, c - pass * ts);
-    r.n0 = (int)rb * 16;
+    r.n0 = (int)(ri * round_blocks + bi) * 16;
     r.nrows = min((int)nblk * 16, m.N - r.n0);
     r.nblk = (int)nblk;
     u += nblk;

@@ -62,7 +62,6 @@ constexpr int kNG = kMaxTS / 8;
 constexpr int kGroupStageBytes = 8 * kKS * 2;  // fp16 tile of one 8-token group x one stage
 constexpr int kActBytes = 64 * 1024;
 constexpr int kStagingBytes = kCW * kMaxTS * 16 * 2;
-constexpr uint64_t kDrainLimitNs = 100000000ull;  // 100 ms
 constexpr uint64_t kActPrefetchMax = 8u << 20;     // activations prefetched into L2 up to 8 MiB
 // 16-byte activation slices per thread in a pass setup: the tile holds
 // kActBytes / 16 slices, spread over the CTA.
@@ -421,7 +420,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int c = 0; c < nst; ++c) {
       const int slot = (int)(consumed % kSlots);
       if (!*abort_flag &&
-          !mbar_wait_bounded(&wfull[slot], (consumed / kSlots) & 1u, kWaitLimitNs))
+          !mbar_wait_bounded(&wfull[slot], (consumed / kSlots) & 1u, p.wait_limit_ns))
         *abort_flag = 1;
       if (!*abort_flag) {
         const uint8_t *sw = wring + slot * kStageW;

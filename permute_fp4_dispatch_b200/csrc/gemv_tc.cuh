@@ -10,12 +10,14 @@
 // Design (taken when experts hold more tokens than a decode pass; the FP4
 // weight stream and its dequantisation bound it):
 //   * Work is expert-major: an active expert's pairs (CSR from
-//     moe_create_indices) are taken in passes of up to kTS = 64 tokens and
-//     each pass sweeps the expert's N rows in 16-row blocks.  The flat list of
-//     (expert, pass, row block) units is split into equal contiguous ranges
-//     cut at round boundaries, one per persistent CTA (grid = SM count).  Consecutive blocks of one
-//     (expert, pass) form a round of up to 128 rows: one tcgen05 MMA tile
-//     (M = 128 weight rows, N = tokens rounded up to 16, fp32 in TMEM).
+//     moe_create_indices) are taken in passes of up to kTS = 64 tokens; the
+//     expert's N rows form rounds of up to 128 rows (8 blocks of 16), and the
+//     units (16-row blocks) are ordered by round, then pass, then block, so
+//     the passes over one round of weights follow each other and re-read it
+//     from L2.  The flat unit list is split into equal contiguous ranges, one
+//     per persistent CTA (grid = SM count).  A round of one pass is one
+//     tcgen05 MMA tile (M = 128 weight rows, N = tokens rounded up to 16,
+//     fp32 in TMEM).
 //   * Warp roles (10 warps):
 //       warp 8      TMA producer: streams each round's FP4 rows and E4M3
 //                   scales in chunks of kKC = 256 columns into a kStages-deep
@@ -74,7 +76,7 @@ constexpr size_t kOffStart = kOffPrefix + (kMaxExperts + 4) * 4;
 constexpr size_t kOffEid = kOffStart + (kMaxExperts + 4) * 4;
 constexpr size_t kOffPair = kOffEid + (kMaxExperts + 4) * 4;     // [2][kTS] pair ids
 constexpr size_t kOffBar = kOffPair + 2 * kTS * 4;
-constexpr int kNumBars = 2 * kStages + 8;
+constexpr int kNumBars = 2 * kStages + 9;
 constexpr size_t kOffMisc = kOffBar + kNumBars * 8;             // tmem slot, abort flag
 constexpr size_t kSmemBytes = kOffMisc + 16 + 1024;             // + alignment slack
 
@@ -98,6 +100,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *a_empty = a_full + 2;       // [2]
   uint64_t *d_full = a_empty + 2;       // [2]
   uint64_t *d_empty = d_full + 2;       // [2]
+  uint64_t *mma_drain = d_empty + 2;    // completes once every MMA issued so far is done
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffMisc);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffMisc + 8);
 
@@ -124,6 +127,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&d_full[b], 1u);
       mbar_init(&d_empty[b], (uint32_t)kDQ);
     }
+    mbar_init(mma_drain, 1u);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -134,15 +138,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tbase = *tmem_slot;
 
   const uint32_t U = prefix[A];
-  uint32_t u_begin, u_end;
-  cta_round_range(U, RB, kBlocksPerRound, u_begin, u_end);
+  // equal contiguous unit ranges (a range may begin or end inside a round)
+  const uint32_t u_begin = muldiv(U, blockIdx.x, gridDim.x);
+  const uint32_t u_end = muldiv(U, blockIdx.x + 1, gridDim.x);
   const int nchunks = (K + kKC - 1) / kKC;
   const int64_t sf_row_bytes = K / 16;
   const Meta meta{prefix, s_start, s_eid, N};
 
   auto wait = [&](uint64_t *bar, uint32_t parity) {
     if (*abort_flag) return;
-    if (!mbar_wait_bounded(bar, parity, kWaitLimitNs)) *abort_flag = 1;
+    if (!mbar_wait_bounded(bar, parity, p.wait_limit_ns)) *abort_flag = 1;
   };
 
   if (warp == kTmaWarp) {
@@ -155,11 +160,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tmap_w);
       if (SF_TMA) prefetch_tmap(&tmap_sf);
     }
+    uint32_t issued = 0;  // stages filled so far (a prefix of the sequence: an abort is final)
     while (iter.next(meta, RB, r)) {
       for (int c = 0; c < nchunks; ++c, ++it) {
         const int s = (int)(it % kStages);
         wait(&empty[s], ((it / kStages) & 1u) ^ 1u);
-        if (*abort_flag) continue;
+        // lane 0's view of the abort flag decides for the whole warp
+        if (__shfl_sync(0xffffffffu, *abort_flag, 0)) continue;
+        issued = it + 1;
         const int k0 = c * kKC;
         uint8_t *sw = smem + (size_t)s * kStageBytes;
         uint8_t *ssf = sw + kStageW;
@@ -175,11 +183,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!SF_TMA) {
           const uint32_t sb = (uint32_t)min(kKC, K - k0) / 16;
           const uint8_t *sbase = p.sfw + ((int64_t)r.e * N + r.n0) * sf_row_bytes + k0 / 16;
-          for (int row = lane; row < r.nrows; row += 32)
-            for (uint32_t q = 0; q < sb; q += 4)
-              cp_async4(ssf + row * kSFStride + q, sbase + row * sf_row_bytes + q);
-          cp_async_mbar_arrive_noinc(&full[s]);
+          if ((sf_row_bytes & 3) == 0) {
+            // 4-byte aligned scale rows (K % 64 == 0): asynchronous copies
+            for (int row = lane; row < r.nrows; row += 32)
+              for (uint32_t q = 0; q < sb; q += 4)
+                cp_async4(ssf + row * kSFStride + q, sbase + row * sf_row_bytes + q);
+            cp_async_mbar_arrive_noinc(&full[s]);
+          } else {
+            // K % 64 == 32: rows are 2-byte aligned; plain loads and stores,
+            // published by this lane's arrival (release semantics)
+            for (int row = lane; row < r.nrows; row += 32)
+              for (uint32_t q = 0; q < sb; q += 2)
+                *reinterpret_cast<uint16_t *>(ssf + row * kSFStride + q) =
+                    __ldg(reinterpret_cast<const uint16_t *>(sbase + row * sf_row_bytes + q));
+            mbar_arrive(&full[s]);
+          }
         }
+      }
+    }
+    // After an abort, let the copies still in flight land before the CTA
+    // exits (bounded again): stage s was filled ceil((issued - s) / kStages) times.
+    if (lane == 0 && *abort_flag) {
+      for (int s = 0; s < kStages; ++s) {
+        const uint32_t fills =
+            issued > (uint32_t)s ? (issued - (uint32_t)s + kStages - 1) / kStages : 0u;
+        if (fills) mbar_wait_bounded(&full[s], (fills - 1) & 1u, kDrainLimitNs);
       }
     }
   } else if (warp == kMmaWarp) {
@@ -215,6 +243,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_commit(&d_full[d]);
         ++rnd;
       }
+      // no MMA may still read shared or tensor memory when the CTA releases them
+      umma_commit(mma_drain);
+      mbar_wait_bounded(mma_drain, 0u, kDrainLimitNs);
     }
     __syncwarp();
   } else {

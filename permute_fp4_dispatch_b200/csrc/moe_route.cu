@@ -17,6 +17,7 @@
 #include "common.cuh"
 #include "create_indices.cuh"
 #include "dispatch_mxfp4.cuh"
+#include "gemv_bs.cuh"
 #include "gemv_mma.cuh"
 #include "gemv_tc.cuh"
 #include "mask.cuh"
@@ -181,6 +182,7 @@ struct LibMaps {
   bool sf_tma = false;  // K % 256 == 0: scale boxes for the tensor-memory variant,
                         // and the line map of the decode variant
   CUtensorMap tw, tsf, tlines, tsf_lines;
+  CUtensorMap tbs;      // block-scaled variant: 128 rows x 128 bytes, 128B swizzle
 };
 constexpr int kMapCache = 8;
 LibMaps g_maps[kMapCache];
@@ -204,9 +206,14 @@ bool library_maps(const uint8_t *w, const uint8_t *sfw, int E, int N, int K, Lib
   std::memset(&m.tsf, 0, sizeof m.tsf);
   std::memset(&m.tlines, 0, sizeof m.tlines);
   std::memset(&m.tsf_lines, 0, sizeof m.tsf_lines);
+  std::memset(&m.tbs, 0, sizeof m.tbs);
   // the tensor-memory variant reads 16-row x 128-byte weight boxes and 16-row x 16-byte scale boxes
   static_assert(moe::gemv::tc::kWStride == 128 && moe::gemv::tc::kSFStride == 16, "box width");
   if (!encode_u8_3d(&m.tw, w, (uint64_t)K / 2, (uint64_t)N, (uint64_t)E, 128, 16,
+                    CU_TENSOR_MAP_SWIZZLE_128B))
+    return false;
+  static_assert(moe::gemv::bs::kATile == 128 * 128, "block-scaled weight box");
+  if (!encode_u8_3d(&m.tbs, w, (uint64_t)K / 2, (uint64_t)N, (uint64_t)E, 128, 128,
                     CU_TENSOR_MAP_SWIZZLE_128B))
     return false;
   if (m.sf_tma && !encode_u8_3d(&m.tsf, sfw, (uint64_t)K / 16, (uint64_t)N, (uint64_t)E, 16, 16,
@@ -452,34 +459,92 @@ moe_status_t moe_quantize_weights_nvfp4(const float *w, int32_t E, int32_t N, in
 }
 
 // ------------------------------------------------------------------ step 4b
+namespace {
+size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// The grouping the GEMV computes for itself when the caller passes only the
+// routing map: the moe_create_indices outputs plus that call's own workspace,
+// carved from the caller's workspace in this order, each 256-byte aligned.
+struct GemvGrouping {
+  uint32_t *order, *start, *restore, *stats;
+  int32_t *eids;
+  void *ci_ws;
+  size_t ci_bytes, total;
+};
+GemvGrouping gemv_grouping_layout(int64_t S, int32_t E, void *base) {
+  GemvGrouping g{};
+  uint8_t *b = static_cast<uint8_t *>(base);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    uint8_t *q = b ? b + off : nullptr;
+    off += round256(bytes);
+    return q;
+  };
+  g.order = reinterpret_cast<uint32_t *>(take((size_t)S * 4));
+  g.restore = reinterpret_cast<uint32_t *>(take((size_t)S * 4));
+  g.start = reinterpret_cast<uint32_t *>(take((size_t)(E + 1) * 4));
+  g.eids = reinterpret_cast<int32_t *>(take((size_t)E * 4));
+  g.stats = reinterpret_cast<uint32_t *>(take(2 * 4));
+  g.ci_bytes = moe_create_indices_workspace_bytes(S, E);
+  g.ci_ws = take(g.ci_bytes);
+  g.total = off;
+  return g;
+}
+}  // namespace
+
+size_t moe_grouped_gemv_workspace_bytes(int32_t M, int32_t top_k, int32_t E) {
+  if (M < 0 || top_k < 1 || E < 1) return 0;
+  return gemv_grouping_layout((int64_t)M * top_k, E, nullptr).total;
+}
+
 moe_status_t moe_grouped_gemv_nvfp4(moe_gemv_mode_t mode, const void *act, const uint8_t *sfa,
-                                    float act_global, int32_t M, int32_t top_k,
-                                    const uint8_t *w, const uint8_t *sfw, const float *w_global,
-                                    int32_t E, int32_t N, int32_t K,
+                                    float act_global, const int64_t *indices, int32_t M,
+                                    int32_t top_k, const uint8_t *w, const uint8_t *sfw,
+                                    const float *w_global, int32_t E, int32_t N, int32_t K,
                                     const uint32_t *token_expert_order,
                                     const uint32_t *expert_start_indices,
                                     const int32_t *expert_ids,
                                     const uint32_t *expert_usage_stats, void *out,
-                                    cudaStream_t s) {
+                                    void *workspace, size_t ws_bytes, cudaStream_t s) {
   using namespace moe::gemv;
   if (mode != MOE_W4A16 && mode != MOE_W4A4) return MOE_ERR_INVALID_ARG;
   if (M < 0 || top_k < 1 || E < 1 || E > kMaxExperts || top_k > E || N < 8 || N % 8 != 0 ||
-      K < 64 || K % 64 != 0 || !(act_global > 0.0f))
+      K < 32 || K % 32 != 0 || !(act_global > 0.0f))
     return MOE_ERR_INVALID_ARG;
-  if (!w || !sfw || !expert_start_indices || !expert_ids || !expert_usage_stats)
-    return MOE_ERR_INVALID_ARG;
-  if (M > 0 && (!act || !out || !token_expert_order)) return MOE_ERR_INVALID_ARG;
+  // the step-2 grouping: all four given, or none (then computed from indices)
+  const int given = (token_expert_order != nullptr) + (expert_start_indices != nullptr) +
+                    (expert_ids != nullptr) + (expert_usage_stats != nullptr);
+  if (given != 0 && given != 4) return MOE_ERR_INVALID_ARG;
+  if (!w || !sfw) return MOE_ERR_INVALID_ARG;
+  if (M > 0 && (!act || !out)) return MOE_ERR_INVALID_ARG;
+  if (given == 0 && M > 0 && !indices) return MOE_ERR_INVALID_ARG;
+  if (!aligned(indices, 8)) return MOE_ERR_INVALID_ARG;
   if (mode == MOE_W4A4 && M > 0 && !sfa) return MOE_ERR_INVALID_ARG;
   if (!aligned(act, 16) || !aligned(w, 16) || !aligned(sfw, 16) || !aligned(out, 16) ||
-      !aligned(w_global, 4))
+      !aligned(w_global, 4) || !aligned(sfa, 4))
     return MOE_ERR_INVALID_ARG;
   // the flat unit count must fit 32 bits: (S / 32 + E) * ceil(N / 16)
   const int64_t S = (int64_t)M * top_k;
   if ((S / 8 + E + 1) * ((N + 15) / 16) >= (int64_t(1) << 32)) return MOE_ERR_INVALID_ARG;
+  if (given == 0 && M > 0) {
+    const GemvGrouping g0 = gemv_grouping_layout(S, E, nullptr);
+    if (!workspace || ws_bytes < g0.total || !aligned(workspace, 256)) return MOE_ERR_WORKSPACE;
+  }
   int sms = 0;
   moe_status_t st = check_device(&sms);
   if (st != MOE_OK) return st;
   if (M == 0) return MOE_OK;
+  if (given == 0) {
+    // group the pairs of the routing map first, into the caller's workspace
+    const GemvGrouping g = gemv_grouping_layout(S, E, workspace);
+    st = moe_create_indices(indices, S, E, g.order, g.start, g.restore, g.eids, g.stats, nullptr,
+                            g.ci_ws, g.ci_bytes, s);
+    if (st != MOE_OK) return st;
+    token_expert_order = g.order;
+    expert_start_indices = g.start;
+    expert_ids = g.eids;
+    expert_usage_stats = g.stats;
+  }
   Params p;
   p.act = act;
   p.sfa = sfa;
@@ -496,19 +561,35 @@ moe_status_t moe_grouped_gemv_nvfp4(moe_gemv_mode_t mode, const void *act, const
   p.eids = expert_ids;
   p.stats = expert_usage_stats;
   p.out = static_cast<uint16_t *>(out);
+  p.wait_limit_ns = kWaitLimitNs;
+  // test hook: MOE_TEST_WAIT_LIMIT_NS shortens every pipeline wait of the GEMV,
+  // so a test can make one expire and check MOE_DEVERR_WAIT_TIMEOUT (the kernel
+  // then winds down and waits for its copies in flight; no fault, no hang)
+  if (const char *v = std::getenv("MOE_TEST_WAIT_LIMIT_NS")) p.wait_limit_ns = std::strtoull(v, nullptr, 10);
   LibMaps maps;
   if (!library_maps(w, sfw, E, N, K, &maps)) return MOE_ERR_CUDA;
-  // Decode-sized passes (no more tokens per expert on average than one pass
-  // of the register-dequant mma.sync variant holds) take that variant; more
-  // tokens per expert take the tensor-memory variant, whose tcgen05 MMA has a
-  // fixed per-instruction cost up to N = 64 and whose passes hold 64 tokens.
+  // W4A4 with K % 64 == 0 runs on the block-scaled FP4 tensor core (no
+  // dequantisation).  W4A16: decode-sized passes (no more tokens per expert on
+  // average than one pass of the register-dequant mma.sync variant holds)
+  // take that variant; more tokens per expert take the tensor-memory variant,
+  // whose tcgen05 MMA has a fixed per-instruction cost up to N = 64 and whose
+  // passes hold 64 tokens.
+  const bool bs_ok = mode == MOE_W4A4 && K % 64 == 0;
+  bool use_bs = bs_ok;
   const int ts_mma = maps.sf_tma ? mma::tokens_per_pass(K) : 0;
   const bool mma_ok = ts_mma >= 8 && E <= mma::kMaxActive;
   bool use_mma = mma_ok && S <= (int64_t)ts_mma * E;
-  // test hook: MOE_GEMV_VARIANT=mma|tc forces a variant (both are exact for every input)
+  // test hook: MOE_GEMV_VARIANT=mma|tc|bs forces a variant where it applies
+  // (every variant is exact for every input it accepts)
   if (const char *v = std::getenv("MOE_GEMV_VARIANT")) {
-    if (v[0] == 'm' && mma_ok) use_mma = true;
-    if (v[0] == 't') use_mma = false;
+    if (v[0] == 'm' && mma_ok) use_mma = true, use_bs = false;
+    if (v[0] == 't') use_mma = false, use_bs = false;
+    if (v[0] == 'b' && bs_ok) use_bs = true;
+  }
+  if (use_bs) {
+    if ((st = set_smem(bs::grouped_gemv_bs_kernel, bs::kSmemBytes)) != MOE_OK) return st;
+    return launch_pdl(bs::grouped_gemv_bs_kernel, dim3((unsigned)sms), dim3(bs::kThreads),
+                      bs::kSmemBytes, s, p, maps.tbs);
   }
   if (use_mma) {
     void (*kern)(const Params, const int, const CUtensorMap, const CUtensorMap) =

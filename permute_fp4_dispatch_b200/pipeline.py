@@ -159,10 +159,11 @@ class RoutingPipeline:
 
     def gemv(self, stream=None):
         act = self.x if self.gemv_mode == MOE_W4A16 else self.xq
-        moe_grouped_gemv_nvfp4(self.gemv_mode, act, self.sfa, self.act_global, self.N,
-                               self.top_k, self.wq, self.sfw, self.w_global, self.E, self.N_out,
-                               self.K, self.token_expert_order, self.expert_start_indices,
-                               self.expert_ids, self.expert_usage_stats, self.expert_out, stream)
+        moe_grouped_gemv_nvfp4(self.gemv_mode, act, self.sfa, self.act_global, self.routing_map,
+                               self.N, self.top_k, self.wq, self.sfw, self.w_global, self.E,
+                               self.N_out, self.K, self.token_expert_order,
+                               self.expert_start_indices, self.expert_ids,
+                               self.expert_usage_stats, self.expert_out, stream=stream)
 
     def combine(self, stream=None):
         moe_combine(self.expert_out, self.router_weights, self.routing_map, self.N, self.top_k,
@@ -229,6 +230,18 @@ class RoutingPipeline:
         here.record(main)
         self._timer.wait_event(here)
         event.record(self._timer)
+
+    def kernel_steps(self):
+        """(name, step) for every launch of one step, in run() order; each step
+        takes the stream to enqueue on.  For per-kernel timing."""
+        steps = [("mask+create_indices", self.mask_and_create_indices)]
+        if self.dispatch:
+            steps.append(("dispatch_mxfp4", self.dispatch_mxfp4))
+        if self.gemv_mode == MOE_W4A4:
+            steps.append(("quant_act_nvfp4", self.quantize_activations))
+        steps.append(("grouped_gemv", self.gemv))
+        steps.append(("combine", self.combine))
+        return steps
 
     def launches_per_run(self) -> int:
         # mask + create_indices: one fused kernel up to 1024 slots, else mask and 1-2 kernels

@@ -82,3 +82,37 @@ def quantize_all_weights(pipe, cfg, chunk: int = 16):
 
 def oracle_weights(cfg, experts):
     return oracle.quantize_weights_nvfp4(wl.expert_weights_f32_many(cfg, experts))
+
+
+def oracle_gemv_rows_threaded(mode, ids, wq, sfw, gw, act_bf16=None, xq=None, sfa=None,
+                              g_a: float = 1.0, rows_per_task: int = 4, threads: int | None = None):
+    """oracle.grouped_gemv over every row of ``ids`` [M, top_k], computed in
+    independent row chunks on a thread pool (the oracle's C code runs with the
+    GIL released).  Same function, same arithmetic per element; only the rows
+    are spread over the host cores."""
+    import os
+    from concurrent.futures import ThreadPoolExecutor
+    M = ids.shape[0]
+    out = np.full((M, ids.shape[1], wq.shape[1]), np.nan)
+    n = threads or max(1, min(32, len(os.sched_getaffinity(0))))
+
+    def run(m0):
+        m1 = min(M, m0 + rows_per_task)
+        kw = {}
+        if act_bf16 is not None:
+            kw["act_bf16"] = act_bf16[m0:m1]
+        if xq is not None:
+            kw["xq"], kw["sfa"] = xq[m0:m1], sfa[m0:m1]
+        out[m0:m1] = oracle.grouped_gemv(mode, ids[m0:m1], wq, sfw, gw, g_a=g_a, **kw)
+
+    with ThreadPoolExecutor(n) as ex:
+        list(ex.map(run, range(0, M, rows_per_task)))
+    return out
+
+
+def decode_passes(ids: np.ndarray, E: int, tokens_per_pass: int) -> int:
+    """(expert, pass) pairs of a routing map when every expert's pairs are
+    taken tokens_per_pass at a time."""
+    valid = ids[(ids >= 0) & (ids < E)]
+    counts = np.bincount(valid, minlength=E)
+    return int(((counts + tokens_per_pass - 1) // tokens_per_pass).sum())

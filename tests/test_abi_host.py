@@ -56,12 +56,21 @@ def test_host_validation_runs_before_any_device_work(lib):
     assert lib.moe_dispatch_mxfp4(P, 4, 48, 2, 4, P, P, P, P, P, 8, P, None) == 1   # K % 32
     assert lib.moe_quantize_activations_nvfp4(P, 4, 24, 1.0, P, P, None) == 1      # K % 16
     assert lib.moe_quantize_activations_nvfp4(P, 4, 32, 0.0, P, P, None) == 1      # g > 0
-    assert lib.moe_grouped_gemv_nvfp4(0, P, None, 1.0, 4, 2, P, P, None, 4, 12, 64,
-                                      P, P, P, P, P, None) == 1                     # N % 8
-    assert lib.moe_grouped_gemv_nvfp4(0, P, None, 1.0, 4, 2, P, P, None, 4, 16, 96,
-                                      P, P, P, P, P, None) == 1                     # K % 64
-    assert lib.moe_grouped_gemv_nvfp4(0, 8 + 1, None, 1.0, 4, 2, P, P, None, 4, 16, 64,
-                                      P, P, P, P, P, None) == 1                     # alignment
+    gemv = lambda *a: lib.moe_grouped_gemv_nvfp4(*a)  # noqa: E731
+    G = (P, P, P, P)                                   # a full step-2 grouping
+    assert gemv(0, P, None, 1.0, P, 4, 2, P, P, None, 4, 12, 64, *G, P, None, 0, None) == 1  # N % 8
+    assert gemv(0, P, None, 1.0, P, 4, 2, P, P, None, 4, 16, 80, *G, P, None, 0, None) == 1  # K % 32
+    assert gemv(0, 8 + 1, None, 1.0, P, 4, 2, P, P, None, 4, 16, 64, *G, P, None, 0,
+                None) == 1                                                            # alignment
+    assert gemv(0, P, None, 1.0, P, 4, 2, P, P, None, 4, 16, 64, P, None, P, P, P, None, 0,
+                None) == 1                                                            # partial grouping
+    assert gemv(0, P, None, 1.0, None, 4, 2, P, P, None, 4, 16, 64, None, None, None, None, P,
+                None, 0, None) == 1                                                   # no map at all
+    ws = moe.moe_grouped_gemv_workspace_bytes(4, 2, 4)
+    assert gemv(0, P, None, 1.0, P, 4, 2, P, P, None, 4, 16, 64, None, None, None, None, P,
+                P * 16, ws - 1, None) == 3                                            # workspace size
+    assert gemv(0, P, None, 1.0, P, 4, 2, P, P, None, 4, 16, 64, None, None, None, None, P,
+                P * 16 + 16, ws, None) == 3                                           # workspace align
     assert lib.moe_combine(P, P, P, 4, 2, 12, 4, 0, 1.0, P, None) == 1              # H % 8
     assert lib.moe_combine(P, P, P, 4, 2, 16, 4, 7, 1.0, P, None) == 1              # epilogue
 
@@ -72,3 +81,12 @@ def test_workspace_sizing(lib):
     assert big == 256 + 12 * 64 * 4
     assert moe.moe_mxfp4_row_stride(2048) == 1088
     assert moe.moe_mxfp4_row_stride(2880) == 1536
+    # grouped GEMV workspace: order, restore [S] u32, starts [E+1], ids [E], stats [2],
+    # then the grouping call's own workspace, each section 256-byte aligned
+    r = lambda n: -(-n // 256) * 256  # noqa: E731
+    S, E = 1024, 128
+    assert moe.moe_grouped_gemv_workspace_bytes(128, 8, 128) == (
+        2 * r(4 * S) + r(4 * (E + 1)) + r(4 * E) + r(8) + 256)
+    S, E = 98304, 64
+    assert moe.moe_grouped_gemv_workspace_bytes(16384, 6, 64) == (
+        2 * r(4 * S) + r(4 * (E + 1)) + r(4 * E) + r(8) + r(256 + 12 * 64 * 4))

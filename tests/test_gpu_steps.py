@@ -282,6 +282,11 @@ GEMV_CASES = [
     # decode-like: K = 2048 (two full stages), about 16 tokens per expert
     ("decode-like", wl.small_config("dlike", N=64, real=64, K=2048, E=16, top_k=4, N_out=136),
      "w4a16"),
+    # K = 32 * odd (K % 64 == 32): 2-byte aligned scale rows, a partial last chunk
+    ("k32odd-w4a16", wl.small_config("k32odd", N=30, real=28, K=224, E=5, top_k=2, N_out=72),
+     "w4a16"),
+    ("k32odd-w4a4", wl.small_config("k32odd", N=30, real=28, K=224, E=5, top_k=2, N_out=72),
+     "w4a4"),
     # activations spanning many binades (per-chunk power-of-two scaling)
     ("wide-range", wl.small_config("wide", N=24, real=24, K=1024, E=6, top_k=2, N_out=128,
                                    outlier_frac=0.05, outlier_mult=3000.0), "w4a16"),
@@ -305,9 +310,11 @@ def run_gemv_case(cfg, mode, act_global=1.0):
     return pipe, x, oracle.mask_padding(ids, cfg.real)
 
 
-@pytest.fixture(params=["auto", "mma", "tc"])
+@pytest.fixture(params=["auto", "mma", "tc", "bs"])
 def gemv_variant(request, monkeypatch):
-    """Run a GEMV case through the host's choice and through each kernel variant."""
+    """Run a GEMV case through the host's choice and through each kernel variant
+    (a variant that does not apply to the case -- the block-scaled one for
+    W4A16, the decode one for K % 256 != 0 -- leaves the host's choice)."""
     if request.param != "auto":
         monkeypatch.setenv("MOE_GEMV_VARIANT", request.param)
     yield request.param
@@ -353,6 +360,61 @@ def test_gemv_token_major_equals_flattened_pairs(gemv_variant):
     flat.gemv()
     np.testing.assert_array_equal(host_bf16_bits(flat.expert_out).reshape(-1),
                                   host_bf16_bits(pipe.expert_out).reshape(-1))
+
+
+def bare_gemv(pipe, cfg, out, ws, stream=None):
+    """The card's call shape: the routing map and a workspace, no grouping."""
+    act = pipe.x if pipe.gemv_mode == moe.MOE_W4A16 else pipe.xq
+    moe.moe_grouped_gemv_nvfp4(pipe.gemv_mode, act, pipe.sfa, pipe.act_global, pipe.routing_map,
+                               cfg.N, cfg.top_k, pipe.wq, pipe.sfw, pipe.w_global, cfg.E,
+                               cfg.N_out, cfg.K, out=out, workspace=ws, ws_bytes=ws.numel(),
+                               stream=stream)
+
+
+@pytest.mark.parametrize("mode", ["w4a16", "w4a4"])
+def test_gemv_from_the_routing_map_alone(mode, gemv_variant):
+    """indices [M, top_k] plus caller workspace and no step-2 grouping gives
+    the same bits as the call that is handed the grouping."""
+    cfg = wl.small_config("bare", N=50, real=44, K=512, E=7, top_k=4, N_out=136)
+    pipe, x, ids = run_gemv_case(cfg, mode)
+    ws = torch.full((moe.moe_grouped_gemv_workspace_bytes(cfg.N, cfg.top_k, cfg.E),), 0x5A,
+                    dtype=torch.uint8, device="cuda")
+    out = torch.empty_like(pipe.expert_out)
+    out.view(torch.int16).fill_(SENTINEL)
+    bare_gemv(pipe, cfg, out, ws)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(host_bf16_bits(out), host_bf16_bits(pipe.expert_out))
+
+
+def test_gemv_from_the_routing_map_follows_graph_replays():
+    """The map is read on the device: a captured call follows new expert ids
+    written between replays."""
+    cfg = wl.small_config("bare_graph", N=40, real=40, K=256, E=6, top_k=2, N_out=64)
+    pipe, x, _ = run_gemv_case(cfg, "w4a16")
+    ws = torch.empty(moe.moe_grouped_gemv_workspace_bytes(cfg.N, cfg.top_k, cfg.E),
+                     dtype=torch.uint8, device="cuda")
+    out = torch.empty_like(pipe.expert_out)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        bare_gemv(pipe, cfg, out, ws, s)              # warm-up outside capture
+    s.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            bare_gemv(pipe, cfg, out, ws, s)
+    wq, sfw, gw = oracle_weights(cfg, range(cfg.E))
+    rng = np.random.default_rng(5)
+    for _ in range(3):
+        ids = np.stack([rng.choice(cfg.E, cfg.top_k, replace=False) for _ in range(cfg.N)])
+        ids[rng.random(ids.shape) < 0.1] = -1        # some slots route nowhere
+        pipe.routing_map.copy_(dev(ids.astype(np.int64)))
+        out.view(torch.int16).fill_(SENTINEL)
+        g.replay()
+        torch.cuda.synchronize()
+        ref = oracle.grouped_gemv("w4a16", ids, wq, sfw, gw, act_bf16=x)
+        routed = ~np.isnan(ref[..., 0])
+        assert np.all(host_bf16_bits(out)[~routed] == SENTINEL)
+        assert_float_parity(host_bf16_f64(out)[routed], ref[routed], what="graph replay")
 
 
 def test_gemv_activation_range_is_reported():
@@ -421,7 +483,8 @@ def test_combine_into_pinned_host_memory():
 # ------------------------------------------------------------------ boundary
 def test_invalid_arguments_launch_nothing():
     with pytest.raises(moe.MoeError) as e:
-        moe.moe_grouped_gemv_nvfp4(0, 16, 0, 1.0, 4, 2, 16, 16, 0, 4, 12, 64, 16, 16, 16, 16, 16)
+        moe.moe_grouped_gemv_nvfp4(0, 16, 0, 1.0, 16, 4, 2, 16, 16, 0, 4, 12, 64, 16, 16, 16, 16,
+                                   16)
     assert e.value.status == 1
     with pytest.raises(moe.MoeError) as e:
         moe.moe_create_indices(16, 8, 4, 16, 16, 16, 16, 16, None, None, 0)
