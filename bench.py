@@ -323,6 +323,32 @@ def dense_flops(cfg, R: int) -> int:
     return 2 * R * cfg.N_out * cfg.K
 
 
+def count_kernel_nodes(graph):
+    """Kernel nodes of a captured CUDA graph (captured with keep_graph=True):
+    the launches one replay makes.  None when the graph cannot be inspected."""
+    try:
+        from cuda.bindings import runtime as rt
+        g = rt.cudaGraph_t(init_value=graph.raw_cuda_graph())
+        err, _, n = rt.cudaGraphGetNodes(g, 0)
+        err, nodes, n = rt.cudaGraphGetNodes(g, n)
+        if err != rt.cudaError_t.cudaSuccess:
+            return None
+        kernel = rt.cudaGraphNodeType.cudaGraphNodeTypeKernel
+        return sum(1 for nd in nodes[:n] if rt.cudaGraphNodeGetType(nd)[1] == kernel)
+    except Exception:
+        return None
+
+
+def describe_step_graph(pipe) -> str:
+    if pipe.order == "gemv_groups":
+        return ("one CUDA graph per step: mask, the GEMV on the routing map (it groups the "
+                "pairs in-kernel) and the combine, chained by programmatic dependent launch; "
+                "create_indices and the MXFP4 dispatch on a stream forked after the mask")
+    return ("one CUDA graph per step: mask + create_indices, GEMV, combine, chained by "
+            "programmatic dependent launch; the MXFP4 dispatch on a stream forked after "
+            "mask + create_indices, beside the GEMV")
+
+
 class L2Flush:
     """Between timed steps: write a buffer larger than L2, which evicts every
     line of the step's inputs and outputs; mode "write+read" then reads
@@ -402,10 +428,14 @@ def measure_workload(cfg, mode, dev, steps, warmup, flush, peaks, weights, headl
     hbm_peak, bf16_peak = peaks["hbm_gbs"], peaks["bf16_tflops"]
 
     # masking is idempotent for a fixed real_token_count, so replays need no map restore
-    graph = torch.cuda.CUDAGraph()
+    graph = torch.cuda.CUDAGraph(keep_graph=True)
     with torch.cuda.stream(stream):
         with torch.cuda.graph(graph, stream=stream):
             pipe.run(stream, side_stream=side)
+    graph.instantiate()
+    launches = count_kernel_nodes(graph)
+    if launches is None:
+        launches = pipe.launches_per_run()
 
     def replay_times(n, g, after=None):
         starts = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
@@ -518,7 +548,8 @@ def measure_workload(cfg, mode, dev, steps, warmup, flush, peaks, weights, headl
                 "h2d_bytes_per_step": h_in.numel(), "d2h_bytes_per_step": h_out.numel() * 2},
         "weights": ("seeded numpy recipe" if weights == "numpy"
                     else "N(0,0.02) from torch's CUDA generator"),
-        "gpu_launches_per_step": pipe.launches_per_run(),
+        "gpu_launches_per_step": launches,
+        "step_graph": describe_step_graph(pipe),
     }
     extras = {"pipe": pipe, "graph": graph, "kgraph": kgraph, "stream": stream, "side": side,
               "bytes": bytes_,
@@ -591,11 +622,9 @@ def run_ours(args, rank, world, local_rank):
         "data": "synthetic (seeded; weights N(0,0.02) quantised to NVFP4 on device)",
         "config": dict(workload_config(cfg, mode, R, A),
                        l2=flush.describe(),
-                       graph=("one CUDA graph per step: mask + create_indices, GEMV, "
-                              "combine, chained by programmatic dependent launch, the "
-                              "dispatch on a stream forked after mask + create_indices, "
-                              "beside the GEMV; the GEMV's launch time from K more steps of "
-                              "the same graph with timing events around it")),
+                       graph=head["step_graph"] + ("; the GEMV's launch time from K more "
+                                                    "steps of the same graph with timing "
+                                                    "events around it")),
         "roofline": {"kernel": "grouped_gemv_nvfp4", "bound": "hbm", "achieved": gemv_gbs,
                      "peak": hbm, "unit": "GB/s", "frac": gemv_gbs / hbm,
                      "traffic": profiled_traffic(cfg.name),
@@ -610,7 +639,7 @@ def run_ours(args, rank, world, local_rank):
                 "ms_per_step": head["e2e"]["us_per_step"] * 1e-3,
                 "h2d_bytes_per_step": head["e2e"]["h2d_bytes_per_step"],
                 "d2h_bytes_per_step": head["e2e"]["d2h_bytes_per_step"]},
-        "gpu_launches": pipe.launches_per_run() * args.steps,
+        "gpu_launches": head["gpu_launches_per_step"] * args.steps,
         "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
     }
     if workloads:

@@ -60,6 +60,13 @@ typedef enum {
 
 typedef enum { MOE_W4A16 = 0, MOE_W4A4 = 1 } moe_gemv_mode_t;
 
+/* Kernel variants of the grouped GEMV (moe_grouped_gemv_plan). */
+typedef enum {
+  MOE_GEMV_DECODE = 0,         /* few tokens per expert: register dequant + mma.sync    */
+  MOE_GEMV_TENSOR_MEMORY = 1,  /* many tokens per expert: dequant into TMEM + tcgen05    */
+  MOE_GEMV_BLOCK_SCALED = 2    /* W4A4, K % 64 == 0: tcgen05 block-scaled FP4 MMA        */
+} moe_gemv_variant_t;
+
 typedef enum {
   MOE_EPI_NONE = 0,     /* no epilogue fused (has_epilogue_fusion = false)    */
   MOE_EPI_IDENTITY = 1, /* fused elementwise epilogue f(v) = v                */
@@ -70,6 +77,9 @@ typedef enum {
 #define MOE_DEVERR_WAIT_TIMEOUT   0x1u /* a pipeline wait in the GEMV expired           */
 #define MOE_DEVERR_RECV_OVERFLOW  0x2u /* dispatch: routed pairs exceed recv_capacity   */
 #define MOE_DEVERR_ACT_RANGE      0x4u /* W4A16 GEMV: an activation exceeds +-65504     */
+#define MOE_DEVERR_LIMIT          0x8u /* an internal table limit was exceeded; the call
+                                          computed nothing (not expected within the
+                                          documented limits)                           */
 
 /* --------------------------------------------------------------------- */
 /* Step 1 -- Megatron-Core "core.transformer.moe.inference_routing_mask_  */
@@ -264,6 +274,17 @@ MOE_API moe_status_t moe_grouped_gemv_nvfp4(moe_gemv_mode_t mode, const void *ac
                                     const int32_t *expert_ids,
                                     const uint32_t *expert_usage_stats, void *out,
                                     void *workspace, size_t ws_bytes, cudaStream_t s);
+
+/* Which variant moe_grouped_gemv_nvfp4 runs for these shapes on the       */
+/* current device, and whether it groups the routing map inside the GEMV   */
+/* kernel when the grouping is not given (*groups_in_kernel = 1: no        */
+/* grouping launch precedes it).  Host-only query, launches nothing.       */
+/* (An interface aid of this library, no counterpart on the pages.)       */
+/* Errors: MOE_ERR_INVALID_ARG as moe_grouped_gemv_nvfp4 for the shapes.   */
+MOE_API moe_status_t moe_grouped_gemv_plan(moe_gemv_mode_t mode, int32_t M, int32_t top_k,
+                                           int32_t E, int32_t N, int32_t K,
+                                           int32_t grouping_given, int32_t *variant,
+                                           int32_t *groups_in_kernel);
 
 /* --------------------------------------------------------------------- */
 /* Step 5 -- MAX "Struct_ep_combine_wait", execute() (weighted sum with  */

@@ -21,19 +21,24 @@ __all__ = [
     "MoeError", "library", "library_path",
     "MOE_W4A16", "MOE_W4A4", "MOE_EPI_NONE", "MOE_EPI_IDENTITY", "MOE_EPI_SCALE",
     "MOE_DEVERR_WAIT_TIMEOUT", "MOE_DEVERR_RECV_OVERFLOW", "MOE_DEVERR_ACT_RANGE",
+    "MOE_DEVERR_LIMIT",
     "moe_mask_padding", "moe_create_indices_workspace_bytes", "moe_create_indices",
     "moe_create_indices_static", "MOE_CREATE_INDICES_STATIC_SCRATCH",
     "moe_mask_and_create_indices",
     "moe_mxfp4_row_stride", "moe_dispatch_mxfp4", "moe_quantize_activations_nvfp4",
+    "MOE_GEMV_DECODE", "MOE_GEMV_TENSOR_MEMORY", "MOE_GEMV_BLOCK_SCALED",
     "moe_quantize_weights_nvfp4", "moe_grouped_gemv_workspace_bytes", "moe_grouped_gemv_nvfp4",
+    "moe_grouped_gemv_plan",
     "moe_combine",
     "moe_status_string", "moe_get_device_error", "moe_version",
 ]
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED_ARCH, MOE_ERR_WORKSPACE, MOE_ERR_CUDA = range(5)
 MOE_W4A16, MOE_W4A4 = 0, 1
+MOE_GEMV_DECODE, MOE_GEMV_TENSOR_MEMORY, MOE_GEMV_BLOCK_SCALED = 0, 1, 2
 MOE_EPI_NONE, MOE_EPI_IDENTITY, MOE_EPI_SCALE = 0, 1, 2
 MOE_DEVERR_WAIT_TIMEOUT, MOE_DEVERR_RECV_OVERFLOW, MOE_DEVERR_ACT_RANGE = 0x1, 0x2, 0x4
+MOE_DEVERR_LIMIT = 0x8
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_HERE, "libmoe_route.so")
@@ -63,6 +68,7 @@ _SIGS = {
     "moe_grouped_gemv_workspace_bytes": ([_I32, _I32, _I32], _SZ),
     "moe_grouped_gemv_nvfp4": ([_I32, _P, _P, _F32, _P, _I32, _I32, _P, _P, _P, _I32, _I32, _I32,
                                 _P, _P, _P, _P, _P, _P, _SZ, _P], _I32),
+    "moe_grouped_gemv_plan": ([_I32, _I32, _I32, _I32, _I32, _I32, _I32, _P, _P], _I32),
     "moe_combine": ([_P, _P, _P, _I32, _I32, _I32, _I32, _I32, _F32, _P, _P], _I32),
     "moe_status_string": ([_I32], ctypes.c_char_p),
     "moe_get_device_error": ([_P, _I32], _I32),
@@ -207,6 +213,16 @@ def moe_grouped_gemv_nvfp4(mode: int, act, sfa, act_global: float, indices, M: i
         _ptr(w_global), E, N, K, _ptr(token_expert_order), _ptr(expert_start_indices),
         _ptr(expert_ids), _ptr(expert_usage_stats), _ptr(out), _ptr(workspace), ws_bytes,
         _stream(stream)), "moe_grouped_gemv_nvfp4")
+
+
+def moe_grouped_gemv_plan(mode: int, M: int, top_k: int, E: int, N: int, K: int,
+                          grouping_given: bool = False) -> tuple[int, bool]:
+    """(variant, groups_in_kernel) that moe_grouped_gemv_nvfp4 uses for these shapes."""
+    v, g = ctypes.c_int32(0), ctypes.c_int32(0)
+    _check(library().moe_grouped_gemv_plan(mode, M, top_k, E, N, K, int(grouping_given),
+                                           ctypes.byref(v), ctypes.byref(g)),
+           "moe_grouped_gemv_plan")
+    return v.value, bool(g.value)
 
 
 def moe_combine(expert_out, router_weights, topk_ids, M: int, top_k: int, H: int, E: int,

@@ -22,9 +22,10 @@
 //   * warps 2-5 (128 threads): per stage, gather the pass's token rows
 //     (128 bytes of codes each) into the 128B-swizzled K-major B tile, and
 //     the stage's scale factors of both operands into shared memory in the
-//     tensor core's 32-row x 16-byte scale layout, all with cp.async (zero
-//     fill past K, past N and past the pass's tokens), arriving on the
-//     stage's barrier when the copies land; they also run the epilogue
+//     tensor core's 32-row x 16-byte scale layout, all with cp.async laid
+//     out so one warp instruction covers whole rows (no copies for rows the
+//     result does not use), arriving on the stage's barrier when the copies
+//     land; they also run the epilogue
 //     (tensor memory -> scale by g_w * g_a -> bf16 -> out) of the previous
 //     unit while the next one streams;
 //   * warp 1, lane 0: owns tensor memory; per stage copies the scale
@@ -240,7 +241,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ================================================================ token tiles, scales, epilogue
     const int t = (int)threadIdx.x - kSW0 * 32;  // 0 .. 127
     const int q = warp & 3;                       // the TMEM lane quadrant this warp may access
-    const int i32 = t & 31, cq = t >> 5;          // scale row i32 + 32 * cq of the stage layout
     const int64_t xrow = K / 2, sfrow = K / 16;
     const uint8_t *xq = static_cast<const uint8_t *>(p.act);
     UnitWalk walk{u0, u1, a0};
@@ -280,15 +280,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t *pairs = s_pair + (rnd & 1u) * kTS;
       if (t < r.ntok) pairs[t] = __ldg(p.order + r.tok0 + t);
       named_bar_sync(1, kSWThreads);
-      // this thread's token row of the B tile, and the rows of its scale words
-      const bool tok_ok = t < r.ntok;
-      const uint8_t *xrow_t = xq + (tok_ok ? (int64_t)(pairs[t] / (uint32_t)p.top_k) * xrow : 0);
-      const int wrow = r.n0 + i32 + 32 * cq;
-      const bool wrow_ok = wrow < N;
-      const uint8_t *sfa_src = p.sfw + ((int64_t)r.e * N + (wrow_ok ? wrow : 0)) * sfrow;
-      const bool tokb_ok = i32 + 32 * cq < r.ntok;
-      const uint8_t *sfb_src =
-          p.sfa + (tokb_ok ? (int64_t)(pairs[i32 + 32 * cq] / (uint32_t)p.top_k) * sfrow : 0);
+      // Copies are laid out so that a warp instruction covers whole rows: 8
+      // lanes per 128-byte token row (4 rows per instruction), 4 lanes per
+      // row's 16 scale bytes of the stage (8 rows per instruction).  Rows the
+      // MMA result does not use -- tokens past the pass, weight rows past N --
+      // are not copied: D row i depends only on A row i, column j only on B row j.
+      const int bj = t & 7, bt0 = t >> 3;        // B: chunk bj of token bt0 + 16 * it
+      const int skk = t & 3, sr0 = t >> 2;       // scales: word skk of row sr0 + 32 * it
       for (int c = 0; c < nst; ++c, ++it) {
         const int s = (int)(it % kStages);
         wait(&empty[s], ((it / kStages) & 1u) ^ 1u);
@@ -296,20 +294,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint8_t *bt = stage(s) + kATile;
           uint8_t *sfa_s = bt + kBTile, *sfb_s = sfa_s + kSFBytes;
           const int kb0 = c * (kKC / 2);
+          const bool bchunk = kb0 + 16 * (bj + 1) <= xrow;
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const bool ok = tok_ok && kb0 + 16 * (j + 1) <= xrow;
-            cp_async16_zfill(bt + t * 128 + ((j ^ (t & 7)) << 4), ok ? xrow_t + kb0 + 16 * j : xq,
-                             ok ? 16u : 0u);
+          for (int i = 0; i < kTS / 16; ++i) {
+            const int tok = bt0 + 16 * i;
+            if (tok < r.ntok && bchunk) {
+              const uint8_t *src = xq + (int64_t)(pairs[tok] / (uint32_t)p.top_k) * xrow + kb0 + 16 * bj;
+              cp_async16_zfill(bt + tok * 128 + ((bj ^ (tok & 7)) << 4), src, 16u);
+            }
           }
+          const int kc = c * (kKC / 16) + 4 * skk;  // first scale byte of MMA skk of the stage
+          if (kc + 4 <= sfrow) {
 #pragma unroll
-          for (int kk = 0; kk < kKSteps; ++kk) {
-            const int kc = c * (kKC / 16) + 4 * kk;  // first scale byte of the MMA's K range
-            const bool kin = kc + 4 <= sfrow;
-            uint8_t *dst = sfa_s + kk * kSFStep + i32 * 16 + cq * 4;
-            cp_async4_zfill(dst, kin && wrow_ok ? sfa_src + kc : p.sfw, kin && wrow_ok ? 4u : 0u);
-            dst = sfb_s + kk * kSFStep + i32 * 16 + cq * 4;
-            cp_async4_zfill(dst, kin && tokb_ok ? sfb_src + kc : p.sfa, kin && tokb_ok ? 4u : 0u);
+            for (int i = 0; i < 4; ++i) {
+              const int row = sr0 + 32 * i;
+              const int off = skk * kSFStep + (row & 31) * 16 + (row >> 5) * 4;
+              if (r.n0 + row < N)
+                cp_async4_zfill(sfa_s + off, p.sfw + ((int64_t)r.e * N + r.n0 + row) * sfrow + kc, 4u);
+              if (row < r.ntok)
+                cp_async4_zfill(sfb_s + off,
+                                p.sfa + (int64_t)(pairs[row] / (uint32_t)p.top_k) * sfrow + kc, 4u);
+            }
           }
         }
         cp_async_mbar_arrive_noinc(&b_full[s]);

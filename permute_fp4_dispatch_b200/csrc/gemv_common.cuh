@@ -28,11 +28,14 @@ struct Params {
   const uint32_t *stats;
   uint16_t *out;            // bf16 [M, top_k, N]
   uint64_t wait_limit_ns;   // limit of each pipeline wait (kWaitLimitNs unless a test shortens it)
+  const int64_t *indices;   // routing map [M, top_k]: read when order == nullptr (the
+  int32_t E;                // kernel then groups the pairs itself)
 };
 
 struct Round {
   int e;
   uint32_t tok0;
+  uint32_t first;  // rank of the pass's first pair within its expert (pass * tokens per pass)
   int ntok;
   int n0;
   int nrows;
@@ -60,11 +63,11 @@ __device__ __forceinline__ int expert_of_unit(const uint32_t *prefix, uint32_t A
 }
 
 // Walks a CTA's unit range round by round; identical in every thread.
-// Within an active expert with c pairs (P = ceil(c / ts) passes) the units
-// (16-row blocks) are ordered by 128-row round, then pass, then block: the
-// passes over one round of weight rows follow each other, so an expert with
-// more tokens than one pass reads each round's weights from HBM once and
-// from L2 for the other passes.  A round is cut short at the range's end.
+// Within an active expert the units (16-row blocks) are ordered by pass, then
+// block: a pass's activations are gathered once per round of up to
+// round_blocks blocks and its blocks follow each other.  (For bf16
+// activations a pass's rows cost more to re-read than a round of FP4
+// weights, so the weights are the operand re-streamed per pass.)
 struct RoundIter {
   uint32_t u, u_end;
   int a;
@@ -74,28 +77,18 @@ struct RoundIter {
     if (u >= u_end) return false;
     while (u >= m.prefix[a + 1]) ++a;
     const uint32_t v = u - m.prefix[a];
+    const uint32_t pass = v / (uint32_t)RB;
+    const uint32_t rb = v % (uint32_t)RB;
+    uint32_t nblk = (uint32_t)RB - rb;
+    if (nblk > round_blocks) nblk = round_blocks;
+    if (nblk > u_end - u) nblk = u_end - u;
     const uint32_t s0 = m.start[a];
     const uint32_t c = m.start[a + 1] - s0;
-    const uint32_t P = (c + ts - 1) / ts;
-    const uint32_t R8 = ((uint32_t)RB + round_blocks - 1) / round_blocks;
-    const uint32_t full = (R8 - 1) * round_blocks * P;  // units of the rounds before the last
-    uint32_t ri, rem, nb;
-    if (v < full) {
-      ri = v / (round_blocks * P);
-      rem = v - ri * round_blocks * P;
-      nb = round_blocks;
-    } else {
-      ri = R8 - 1;
-      rem = v - full;
-      nb = (uint32_t)RB - ri * round_blocks;
-    }
-    const uint32_t pass = rem / nb, bi = rem % nb;
-    uint32_t nblk = nb - bi;
-    if (nblk > u_end - u) nblk = u_end - u;
     r.e = m.eid[a];
-    r.tok0 = s0 + pass * ts;
-    r.ntok = (int)min(ts, c - pass * ts);
-    r.n0 = (int)(ri * round_blocks + bi) * 16;
+    r.first = pass * ts;
+    r.tok0 = s0 + r.first;
+    r.ntok = (int)min(ts, c - r.first);
+    r.n0 = (int)rb * 16;
     r.nrows = min((int)nblk * 16, m.N - r.n0);
     r.nblk = (int)nblk;
     u += nblk;

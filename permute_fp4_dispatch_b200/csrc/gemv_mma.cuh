@@ -76,12 +76,24 @@ constexpr size_t kOffPrefix = kOffStaging + kStagingBytes;
 constexpr size_t kOffStart = kOffPrefix + (kMaxActive + 4) * 4;
 constexpr size_t kOffEid = kOffStart + (kMaxActive + 4) * 4;
 constexpr size_t kOffPair = kOffEid + (kMaxActive + 4) * 4;
-constexpr size_t kOffBar = kOffPair + kMaxTS * 4;
+// In-kernel grouping (routing map given, no step-2 outputs): every CTA
+// histograms the map and compacts the token lists of the passes in its own
+// range.  With at most kFusedSlots slots and kMaxActive experts there are at
+// most S/16 + E <= 768 passes and a CTA's round-aligned range touches at most
+// ceil(768 / 148) + 1 = 7 of them (one when there are no more passes than CTAs).
+constexpr int kFusedSlots = 4096;
+constexpr int kFusedPer = kFusedSlots / kThreads;  // slots per thread
+constexpr int kMaxCtaPasses = 16;
+constexpr size_t kOffPasses = kOffPair + kMaxTS * 4;                 // [kMaxCtaPasses][kMaxTS]
+constexpr size_t kOffPassMeta = kOffPasses + (size_t)kMaxCtaPasses * kMaxTS * 4;  // [3][kMaxCtaPasses]
+constexpr size_t kOffBar = kOffPassMeta + (size_t)3 * kMaxCtaPasses * 4 + 8;
 constexpr size_t kOffMisc = kOffBar + (size_t)kCW * kSlots * 8;
 constexpr size_t kSmemBytes = kOffMisc + 16 + 1024;
 static_assert(kStageW % 1024 == 0, "stages must keep the 1024-byte swizzle alignment");
 static_assert(kOffBar % 8 == 0, "mbarrier alignment");
 static_assert(kSmemBytes <= 232448, "shared memory per block");
+static_assert(kMaxActive <= kThreads && kStagingBytes >= (kMaxActive + 64) * 4,
+              "the in-kernel grouping keeps one expert per thread and its counters in staging");
 
 // Tokens per pass for a hidden size K (a multiple of 256): as many 8-token
 // groups (up to 2) as the activation tile holds for the whole K; 0 when not
@@ -175,6 +187,7 @@ struct RoundWalk {
     if (nblk > kCW) nblk = kCW;
     if ((uint32_t)nblk > u_end - u) nblk = (int)(u_end - u);
     r.e = m.eid[a];
+    r.first = first;
     r.tok0 = s0 + first;
     r.ntok = (int)min(ts, c - first);
     r.n0 = rb * 16;
@@ -241,13 +254,46 @@ __global__ void __launch_bounds__(kThreads, 1)
   pdl_launch_dependents();
   const int N = p.N, K = p.K;
   const int RB = (N + 15) / 16;
-  const uint32_t A = p.stats[1];
-
-  // the grouping of the active experts (at most kMaxActive, checked on the host)
-  // stays in shared memory: every round looks it up
-  for (uint32_t i = threadIdx.x; i <= A; i += blockDim.x) {
-    s_start[i] = p.start[i];
-    if (i < A) s_eid[i] = p.eids[i];
+  const bool fused = p.order == nullptr;
+  uint32_t *cnt = reinterpret_cast<uint32_t *>(staging);   // prologue only: expert counters
+  uint32_t *scan_scratch = cnt + kMaxActive;               // and block-scan scratch
+  int32_t my_ids[kFusedPer];  // in-kernel grouping: experts of this thread's slots (-1: none)
+  const int fq = fused ? (p.M * p.top_k + kThreads - 1) / kThreads : 0;
+  uint32_t A;
+  if (fused) {
+    // group the routing map here: counts per expert, then the active experts in
+    // ascending id with their CSR offsets (the moe_create_indices definition)
+    const int S = p.M * p.top_k;
+    for (int e = threadIdx.x; e < p.E; e += kThreads) cnt[e] = 0u;
+#pragma unroll
+    for (int j = 0; j < kFusedPer; ++j) {
+      const int slot = (int)threadIdx.x * fq + j;
+      const int64_t id = (j < fq && slot < S) ? __ldg(p.indices + slot) : -1;
+      my_ids[j] = (id >= 0 && id < p.E) ? (int32_t)id : -1;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < kFusedPer; ++j)
+      if (my_ids[j] >= 0) atomicAdd(&cnt[my_ids[j]], 1u);
+    __syncthreads();
+    const uint32_t c = (int)threadIdx.x < p.E ? cnt[threadIdx.x] : 0u;
+    uint32_t n_active, n_routed;
+    const uint32_t pos = block_exclusive_scan(c > 0u ? 1u : 0u, scan_scratch, &n_active);
+    const uint32_t off = block_exclusive_scan(c, scan_scratch, &n_routed);
+    if (c > 0u) {
+      s_eid[pos] = (int32_t)threadIdx.x;
+      s_start[pos] = off;
+    }
+    if (threadIdx.x == 0) s_start[n_active] = n_routed;
+    A = n_active;
+  } else {
+    A = p.stats[1];
+    // the grouping of the active experts (at most kMaxActive, checked on the host)
+    // stays in shared memory: every round looks it up
+    for (uint32_t i = threadIdx.x; i <= A; i += blockDim.x) {
+      s_start[i] = p.start[i];
+      if (i < A) s_eid[i] = p.eids[i];
+    }
   }
   __syncthreads();
   if (warp == 0) {
@@ -267,6 +313,56 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nst = (K + kKS - 1) / kKS;  // stages per block
   const int lines_total = K / 256;
   const Meta meta{prefix, s_start, s_eid, N};
+  uint32_t *s_passes = reinterpret_cast<uint32_t *>(smem + kOffPasses);
+  int n_passes = 0;
+  if (fused) {
+    // token lists of the passes in this CTA's range: pass i of expert e holds
+    // the pairs of rank [first, first + ntok) among e's pairs in ascending
+    // pair order (stable), found with one block scan per distinct expert.
+    // First the distinct passes of the range, in order (one thread).
+    int32_t *pe = reinterpret_cast<int32_t *>(smem + kOffPassMeta);
+    uint32_t *pf = reinterpret_cast<uint32_t *>(pe + kMaxCtaPasses);
+    int32_t *pn = reinterpret_cast<int32_t *>(pf + kMaxCtaPasses);
+    int32_t *s_np = pn + kMaxCtaPasses;
+    if (threadIdx.x == 0) {
+      RoundWalk w;
+      w.init(meta, A, RB, u_begin, u_end);
+      Round rr;
+      int cnt_p = 0, prev_e = -1;
+      uint32_t prev_first = 0xFFFFFFFFu;
+      while (cnt_p < kMaxCtaPasses && w.next(meta, RB, (uint32_t)ts, rr)) {
+        if (rr.e == prev_e && rr.first == prev_first) continue;
+        pe[cnt_p] = rr.e;
+        pf[cnt_p] = rr.first;
+        pn[cnt_p] = rr.ntok;
+        ++cnt_p;
+        prev_e = rr.e;
+        prev_first = rr.first;
+      }
+      *s_np = cnt_p;
+    }
+    __syncthreads();
+    const int np = *s_np;
+    n_passes = np;
+    for (int i = 0; i < np; ++i) {
+      if (i > 0 && pe[i] == pe[i - 1]) continue;  // the passes of one expert share a scan
+      const int e = pe[i];
+      uint32_t mine = 0, total;
+#pragma unroll
+      for (int j = 0; j < kFusedPer; ++j) mine += my_ids[j] == e ? 1u : 0u;
+      uint32_t rank = block_exclusive_scan(mine, scan_scratch, &total);
+#pragma unroll
+      for (int j = 0; j < kFusedPer; ++j) {
+        if (my_ids[j] != e) continue;
+        for (int k = i; k < np && pe[k] == e; ++k)
+          if (rank - pf[k] < (uint32_t)pn[k])
+            s_passes[k * kMaxTS + (rank - pf[k])] = (uint32_t)threadIdx.x * (uint32_t)fq + (uint32_t)j;
+        ++rank;
+      }
+    }
+    __syncthreads();
+  }
+  int pass_idx = -1;  // index of the current pass in s_passes
   uint8_t *wring = smem + kOffW + (size_t)warp * kSlots * kStageW;
   uint8_t *sring = smem + kOffSF + (size_t)warp * kSlots * kStageSF;
   uint64_t *wfull = full + warp * kSlots;
@@ -335,8 +431,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint4 v[kSetupTasks];
       uint32_t sv[kSetupTasks];
       uint32_t my_pair = 0, my_row = 0;
-      if (lane < r.ntok) {
-        my_pair = __ldg(p.order + r.tok0 + lane);
+      ++pass_idx;
+      // (the host's limits keep a CTA's passes within the table; should one
+      // not be, the call reports it and computes nothing rather than read past)
+      const bool listed = !fused || pass_idx < n_passes;
+      if (!listed && threadIdx.x == 0) {
+        raise_device_error(MOE_DEVERR_LIMIT);
+        *abort_flag = 1;
+      }
+      if (lane < r.ntok && listed) {
+        my_pair = fused ? s_passes[pass_idx * kMaxTS + lane] : __ldg(p.order + r.tok0 + lane);
         my_row = my_pair / (uint32_t)p.top_k;
       }
       int tau = tau0, kk = kk0;

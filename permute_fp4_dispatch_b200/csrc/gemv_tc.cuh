@@ -10,14 +10,13 @@
 // Design (taken when experts hold more tokens than a decode pass; the FP4
 // weight stream and its dequantisation bound it):
 //   * Work is expert-major: an active expert's pairs (CSR from
-//     moe_create_indices) are taken in passes of up to kTS = 64 tokens; the
-//     expert's N rows form rounds of up to 128 rows (8 blocks of 16), and the
-//     units (16-row blocks) are ordered by round, then pass, then block, so
-//     the passes over one round of weights follow each other and re-read it
-//     from L2.  The flat unit list is split into equal contiguous ranges, one
-//     per persistent CTA (grid = SM count).  A round of one pass is one
-//     tcgen05 MMA tile (M = 128 weight rows, N = tokens rounded up to 16,
-//     fp32 in TMEM).
+//     moe_create_indices) are taken in passes of up to kTS = 64 tokens and
+//     each pass sweeps the expert's N rows in 16-row blocks.  The flat list of
+//     (expert, pass, row block) units is split into equal contiguous ranges
+//     cut at round boundaries, one per persistent CTA (grid = SM count).
+//     Consecutive blocks of one (expert, pass) form a round of up to 128
+//     rows: one tcgen05 MMA tile (M = 128 weight rows, N = tokens rounded up
+//     to 16, fp32 in TMEM).
 //   * Warp roles (10 warps):
 //       warp 8      TMA producer: streams each round's FP4 rows and E4M3
 //                   scales in chunks of kKC = 256 columns into a kStages-deep
@@ -138,9 +137,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tbase = *tmem_slot;
 
   const uint32_t U = prefix[A];
-  // equal contiguous unit ranges (a range may begin or end inside a round)
-  const uint32_t u_begin = muldiv(U, blockIdx.x, gridDim.x);
-  const uint32_t u_end = muldiv(U, blockIdx.x + 1, gridDim.x);
+  uint32_t u_begin, u_end;
+  cta_round_range(U, RB, kBlocksPerRound, u_begin, u_end);
   const int nchunks = (K + kKC - 1) / kKC;
   const int64_t sf_row_bytes = K / 16;
   const Meta meta{prefix, s_start, s_eid, N};

@@ -492,6 +492,43 @@ GemvGrouping gemv_grouping_layout(int64_t S, int32_t E, void *base) {
 }
 }  // namespace
 
+namespace {
+// Which kernel variant a GEMV call runs, and whether it groups the routing map
+// itself.  W4A4 with K % 64 == 0 runs on the block-scaled FP4 tensor core (no
+// dequantisation).  W4A16 (and W4A4 otherwise): decode-sized passes (no more
+// tokens per expert on average than one pass of the register-dequant
+// mma.sync variant holds) take that variant; more tokens per expert take the
+// tensor-memory variant, whose tcgen05 MMA has a fixed per-instruction cost up
+// to N = 64 and whose passes hold 64 tokens.  Only the decode variant groups
+// a small routing map in-kernel (every CTA histograms the map and compacts the
+// token lists of its own passes); the bound on passes per CTA behind that path
+// needs at most kFusedSlots slots, kMaxActive experts and a full grid.
+struct GemvPlan {
+  moe_gemv_variant_t variant;
+  bool groups_in_kernel;
+};
+GemvPlan plan_gemv(moe_gemv_mode_t mode, int64_t S, int32_t E, int32_t K, bool grouping_given,
+                   int sms) {
+  namespace mma = moe::gemv::mma;
+  const bool bs_ok = mode == MOE_W4A4 && K % 64 == 0;
+  const int ts_mma = K % 256 == 0 ? mma::tokens_per_pass(K) : 0;
+  const bool mma_ok = ts_mma >= 8 && E <= mma::kMaxActive;
+  bool use_bs = bs_ok;
+  bool use_mma = !bs_ok && mma_ok && S <= (int64_t)ts_mma * E;
+  // test hook: MOE_GEMV_VARIANT=mma|tc|bs forces a variant where it applies
+  // (every variant is exact for every input it accepts)
+  if (const char *v = std::getenv("MOE_GEMV_VARIANT")) {
+    if (v[0] == 'm' && mma_ok) use_mma = true, use_bs = false;
+    if (v[0] == 't') use_mma = false, use_bs = false;
+    if (v[0] == 'b' && bs_ok) use_bs = true, use_mma = false;
+  }
+  GemvPlan g;
+  g.variant = use_bs ? MOE_GEMV_BLOCK_SCALED : use_mma ? MOE_GEMV_DECODE : MOE_GEMV_TENSOR_MEMORY;
+  g.groups_in_kernel = !grouping_given && use_mma && S <= mma::kFusedSlots && sms >= 148;
+  return g;
+}
+}  // namespace
+
 size_t moe_grouped_gemv_workspace_bytes(int32_t M, int32_t top_k, int32_t E) {
   if (M < 0 || top_k < 1 || E < 1) return 0;
   return gemv_grouping_layout((int64_t)M * top_k, E, nullptr).total;
@@ -534,7 +571,9 @@ moe_status_t moe_grouped_gemv_nvfp4(moe_gemv_mode_t mode, const void *act, const
   moe_status_t st = check_device(&sms);
   if (st != MOE_OK) return st;
   if (M == 0) return MOE_OK;
-  if (given == 0) {
+  const GemvPlan plan = plan_gemv(mode, S, E, K, given == 4, sms);
+  const bool fused_grouping = plan.groups_in_kernel;
+  if (given == 0 && !fused_grouping) {
     // group the pairs of the routing map first, into the caller's workspace
     const GemvGrouping g = gemv_grouping_layout(S, E, workspace);
     st = moe_create_indices(indices, S, E, g.order, g.start, g.restore, g.eids, g.stats, nullptr,
@@ -561,6 +600,8 @@ moe_status_t moe_grouped_gemv_nvfp4(moe_gemv_mode_t mode, const void *act, const
   p.eids = expert_ids;
   p.stats = expert_usage_stats;
   p.out = static_cast<uint16_t *>(out);
+  p.indices = indices;
+  p.E = E;
   p.wait_limit_ns = kWaitLimitNs;
   // test hook: MOE_TEST_WAIT_LIMIT_NS shortens every pipeline wait of the GEMV,
   // so a test can make one expire and check MOE_DEVERR_WAIT_TIMEOUT (the kernel
@@ -568,24 +609,9 @@ moe_status_t moe_grouped_gemv_nvfp4(moe_gemv_mode_t mode, const void *act, const
   if (const char *v = std::getenv("MOE_TEST_WAIT_LIMIT_NS")) p.wait_limit_ns = std::strtoull(v, nullptr, 10);
   LibMaps maps;
   if (!library_maps(w, sfw, E, N, K, &maps)) return MOE_ERR_CUDA;
-  // W4A4 with K % 64 == 0 runs on the block-scaled FP4 tensor core (no
-  // dequantisation).  W4A16: decode-sized passes (no more tokens per expert on
-  // average than one pass of the register-dequant mma.sync variant holds)
-  // take that variant; more tokens per expert take the tensor-memory variant,
-  // whose tcgen05 MMA has a fixed per-instruction cost up to N = 64 and whose
-  // passes hold 64 tokens.
-  const bool bs_ok = mode == MOE_W4A4 && K % 64 == 0;
-  bool use_bs = bs_ok;
-  const int ts_mma = maps.sf_tma ? mma::tokens_per_pass(K) : 0;
-  const bool mma_ok = ts_mma >= 8 && E <= mma::kMaxActive;
-  bool use_mma = mma_ok && S <= (int64_t)ts_mma * E;
-  // test hook: MOE_GEMV_VARIANT=mma|tc|bs forces a variant where it applies
-  // (every variant is exact for every input it accepts)
-  if (const char *v = std::getenv("MOE_GEMV_VARIANT")) {
-    if (v[0] == 'm' && mma_ok) use_mma = true, use_bs = false;
-    if (v[0] == 't') use_mma = false, use_bs = false;
-    if (v[0] == 'b' && bs_ok) use_bs = true;
-  }
+  const bool use_bs = plan.variant == MOE_GEMV_BLOCK_SCALED;
+  const bool use_mma = plan.variant == MOE_GEMV_DECODE;
+  const int ts_mma = use_mma ? mma::tokens_per_pass(K) : 0;
   if (use_bs) {
     if ((st = set_smem(bs::grouped_gemv_bs_kernel, bs::kSmemBytes)) != MOE_OK) return st;
     return launch_pdl(bs::grouped_gemv_bs_kernel, dim3((unsigned)sms), dim3(bs::kThreads),
@@ -609,6 +635,22 @@ moe_status_t moe_grouped_gemv_nvfp4(moe_gemv_mode_t mode, const void *act, const
   if ((st = set_smem(kern, tc::kSmemBytes)) != MOE_OK) return st;
   return launch_pdl(kern, dim3((unsigned)sms), dim3(tc::kThreads), tc::kSmemBytes, s, p, maps.tw,
                     maps.tsf);
+}
+
+moe_status_t moe_grouped_gemv_plan(moe_gemv_mode_t mode, int32_t M, int32_t top_k, int32_t E,
+                                   int32_t N, int32_t K, int32_t grouping_given,
+                                   int32_t *variant, int32_t *groups_in_kernel) {
+  if (mode != MOE_W4A16 && mode != MOE_W4A4) return MOE_ERR_INVALID_ARG;
+  if (M < 0 || top_k < 1 || E < 1 || E > moe::gemv::kMaxExperts || top_k > E || N < 8 ||
+      N % 8 != 0 || K < 32 || K % 32 != 0 || !variant || !groups_in_kernel)
+    return MOE_ERR_INVALID_ARG;
+  int sms = 0;
+  moe_status_t st = check_device(&sms);
+  if (st != MOE_OK) return st;
+  const GemvPlan g = plan_gemv(mode, (int64_t)M * top_k, E, K, grouping_given != 0, sms);
+  *variant = (int32_t)g.variant;
+  *groups_in_kernel = g.groups_in_kernel ? 1 : 0;
+  return MOE_OK;
 }
 
 // ------------------------------------------------------------------ step 5

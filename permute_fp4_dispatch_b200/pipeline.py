@@ -17,7 +17,8 @@ import torch
 
 from . import (MOE_EPI_IDENTITY, MOE_EPI_NONE, MOE_EPI_SCALE, MOE_W4A4, MOE_W4A16,
                moe_combine, moe_create_indices, moe_create_indices_workspace_bytes,
-               moe_mask_and_create_indices,
+               moe_mask_and_create_indices, moe_grouped_gemv_plan,
+               moe_grouped_gemv_workspace_bytes,
                moe_dispatch_mxfp4, moe_grouped_gemv_nvfp4, moe_mask_padding,
                moe_mxfp4_row_stride, moe_quantize_activations_nvfp4, moe_quantize_weights_nvfp4)
 
@@ -44,9 +45,10 @@ def _arena_views(buf: torch.Tensor, entries):
 
 
 class RoutingPipeline:
-    # where run() forks the MXFP4 dispatch onto side_stream: "routing" (after
-    # mask + create_indices, beside the GEMV, on SMs its CTAs leave free) or
-    # "gemv" (after the GEMV, beside the combine)
+    # where run() forks the MXFP4 dispatch onto side_stream in the
+    # "routing_first" order: "routing" (after mask + create_indices, beside the
+    # GEMV, on SMs its CTAs leave free) or "gemv" (after the GEMV, beside the
+    # combine)
     dispatch_fork = "routing"
 
     def __init__(self, N: int, K: int, E: int, top_k: int, N_out: int, mode: str = "w4a16",
@@ -101,6 +103,19 @@ class RoutingPipeline:
         else:
             self.xq = self.sfa = None
         self.expert_out = torch.zeros((N, top_k, N_out), dtype=torch.bfloat16, device=dev)
+        # the GEMV's own grouping workspace (used when it is handed the map alone)
+        self.gemv_ws_bytes = moe_grouped_gemv_workspace_bytes(N, top_k, E)
+        self.gemv_ws = torch.empty(max(self.gemv_ws_bytes, 256), dtype=u8, device=dev)
+        # Step order of run():
+        #   "gemv_groups"   mask -> GEMV on the routing map (the GEMV groups the
+        #                   pairs in-kernel) -> combine; create_indices and the
+        #                   dispatch on the side stream
+        #   "routing_first" mask + create_indices -> GEMV on the grouping ->
+        #                   combine; the dispatch on the side stream
+        # The first is taken when the GEMV variant for these shapes groups the
+        # map itself (decode-sized W4A16), so grouping is off its critical path.
+        _, in_kernel = moe_grouped_gemv_plan(self.gemv_mode, N, top_k, E, N_out, K)
+        self.order = "gemv_groups" if in_kernel else "routing_first"
         # step 5
         self.output = torch.empty((N, N_out), dtype=torch.bfloat16, device=dev)
         # timing events go on a side stream, so no event sits between two kernels
@@ -158,6 +173,7 @@ class RoutingPipeline:
                                        self.sfa, stream)
 
     def gemv(self, stream=None):
+        """The GEMV on the step-2 grouping."""
         act = self.x if self.gemv_mode == MOE_W4A16 else self.xq
         moe_grouped_gemv_nvfp4(self.gemv_mode, act, self.sfa, self.act_global, self.routing_map,
                                self.N, self.top_k, self.wq, self.sfw, self.w_global, self.E,
@@ -165,25 +181,69 @@ class RoutingPipeline:
                                self.expert_start_indices, self.expert_ids,
                                self.expert_usage_stats, self.expert_out, stream=stream)
 
+    def gemv_on_map(self, stream=None):
+        """The GEMV on the routing map alone (it groups the pairs itself)."""
+        act = self.x if self.gemv_mode == MOE_W4A16 else self.xq
+        moe_grouped_gemv_nvfp4(self.gemv_mode, act, self.sfa, self.act_global, self.routing_map,
+                               self.N, self.top_k, self.wq, self.sfw, self.w_global, self.E,
+                               self.N_out, self.K, out=self.expert_out, workspace=self.gemv_ws,
+                               ws_bytes=self.gemv_ws_bytes, stream=stream)
+
     def combine(self, stream=None):
         moe_combine(self.expert_out, self.router_weights, self.routing_map, self.N, self.top_k,
                     self.N_out, self.E, self.epi, self.alpha, self.output, stream)
 
     def run(self, stream=None, gemv_events=None, side_stream=None, x_ready=None):
-        """All steps in order.  ``gemv_events`` = (start, end) CUDA events
-        recorded around the GEMV launch (from a side stream), for per-kernel
-        timing.  With ``side_stream``, the MXFP4 dispatch (whose buffer neither
-        the GEMV nor the combine reads) runs there and joins at the end.  By
-        default (``dispatch_fork = "routing"``) it forks right after mask +
-        create_indices behind an event-record node, so it starts only once the
-        routing kernel is done: the GEMV's CTAs, launched early by the
-        programmatic dependency, hold the SMs first, and the dispatch runs on
-        the SMs they leave free, finishing before the GEMV does.  With
-        ``"gemv"`` it forks after the GEMV, beside the combine.  ``x_ready`` (a
-        CUDA event) holds back the steps that read the activations --
-        dispatch, activation quantisation, GEMV -- until x has arrived; mask
-        and create_indices run before it."""
+        """All steps in order (see ``order``).  ``gemv_events`` = (start, end)
+        CUDA events recorded around the GEMV launch (from a side stream), for
+        per-kernel timing.  With ``side_stream``, the work whose outputs neither
+        the GEMV nor the combine reads -- the MXFP4 dispatch, and in the
+        "gemv_groups" order create_indices too -- runs there and joins at the
+        end.  ``x_ready`` (a CUDA event) holds back the steps that read the
+        activations -- dispatch, activation quantisation, GEMV -- until x has
+        arrived; mask and create_indices run before it."""
         main = stream if stream is not None else torch.cuda.current_stream()
+        if self.order == "gemv_groups":
+            self._run_gemv_groups(main, gemv_events, side_stream, x_ready)
+        else:
+            self._run_routing_first(main, gemv_events, side_stream, x_ready)
+        if gemv_events is not None:
+            timer_done = torch.cuda.Event()
+            timer_done.record(self._timer)
+            main.wait_event(timer_done)
+
+    def _run_gemv_groups(self, main, gemv_events, side_stream, x_ready):
+        self.mask(main)
+        join = None
+        if side_stream is not None:
+            fork = torch.cuda.Event()
+            fork.record(main)
+            side_stream.wait_event(fork)
+            self.create_indices(side_stream)
+            if self.dispatch:
+                if x_ready is not None:
+                    side_stream.wait_event(x_ready)
+                self.dispatch_mxfp4(side_stream)
+            join = torch.cuda.Event()
+            join.record(side_stream)
+        else:
+            self.create_indices(main)
+        if x_ready is not None:
+            main.wait_event(x_ready)
+        if side_stream is None and self.dispatch:
+            self.dispatch_mxfp4(main)
+        if self.gemv_mode == MOE_W4A4:
+            self.quantize_activations(main)
+        if gemv_events is not None:
+            self._mark(main, gemv_events[0])
+        self.gemv_on_map(main)
+        if gemv_events is not None:
+            self._mark(main, gemv_events[1])
+        self.combine(main)
+        if join is not None:
+            main.wait_event(join)
+
+    def _run_routing_first(self, main, gemv_events, side_stream, x_ready):
         self.mask_and_create_indices(main)
         forked = self.dispatch and side_stream is not None
         early = forked and self.dispatch_fork == "routing"
@@ -218,10 +278,6 @@ class RoutingPipeline:
         self.combine(main)
         if forked:
             main.wait_event(join)
-        if gemv_events is not None:
-            timer_done = torch.cuda.Event()
-            timer_done.record(self._timer)
-            main.wait_event(timer_done)
 
     def _mark(self, main, event):
         """Record ``event`` once everything enqueued on ``main`` so far has run,
@@ -232,20 +288,30 @@ class RoutingPipeline:
         event.record(self._timer)
 
     def kernel_steps(self):
-        """(name, step) for every launch of one step, in run() order; each step
-        takes the stream to enqueue on.  For per-kernel timing."""
-        steps = [("mask+create_indices", self.mask_and_create_indices)]
+        """(name, step) for every step of run(), in order, serialised on one
+        stream; each step takes the stream to enqueue on.  For per-kernel
+        timing."""
+        if self.order == "gemv_groups":
+            steps = [("mask", self.mask), ("create_indices", self.create_indices)]
+        else:
+            steps = [("mask+create_indices", self.mask_and_create_indices)]
         if self.dispatch:
             steps.append(("dispatch_mxfp4", self.dispatch_mxfp4))
         if self.gemv_mode == MOE_W4A4:
             steps.append(("quant_act_nvfp4", self.quantize_activations))
-        steps.append(("grouped_gemv", self.gemv))
+        gemv = self.gemv_on_map if self.order == "gemv_groups" else self.gemv
+        steps.append(("grouped_gemv", gemv))
         steps.append(("combine", self.combine))
         return steps
 
     def launches_per_run(self) -> int:
-        # mask + create_indices: one fused kernel up to 1024 slots, else mask and 1-2 kernels
-        front = 1 if self.S <= 1024 else 1 + (1 if self.S <= 16384 else 2)
-        n = front + (1 if self.dispatch else 0)
+        """Kernel launches of one run() (an estimate; bench.py counts the
+        kernel nodes of the captured graph)."""
+        ci = 1 if self.S <= 16384 else 2
+        if self.order == "gemv_groups":
+            n = 1 + ci + 1                       # mask, create_indices, GEMV (groups in-kernel)
+        else:
+            n = (1 if self.S <= 1024 else 1 + ci) + 1
+        n += 1 if self.dispatch else 0
         n += 1 if self.gemv_mode == MOE_W4A4 else 0
-        return n + 2
+        return n + 1                             # combine

@@ -149,16 +149,19 @@ def test_pipeline_repeatable_bitwise():
             assert torch.equal(a.view(torch.uint8), b.view(torch.uint8))
 
 
-@pytest.mark.parametrize("fork", ["gemv", "routing"])
+@pytest.mark.parametrize("order,fork", [("routing_first", "gemv"), ("routing_first", "routing"),
+                                        ("gemv_groups", None)])
 @pytest.mark.parametrize("mode", ["w4a16", "w4a4"])
-def test_forked_dispatch_graph_matches_sequential(mode, fork):
-    """Dispatch on a forked stream inside a captured graph (forked after the
-    GEMV or after the routing kernel) gives the same bytes as the one-stream
-    order, for every step's output."""
+def test_forked_dispatch_graph_matches_sequential(mode, order, fork):
+    """The side-stream work (dispatch; create_indices too in the gemv_groups
+    order) inside a captured graph gives the same bytes as the one-stream
+    order, for every step's output, in both step orders."""
     cfg = wl.config("decode_30b_a3b")
     x, ids, rw = wl.activations_bf16(cfg), wl.routing(cfg), wl.router_weights(cfg)
     pipe = make_pipeline(cfg, mode)
-    pipe.dispatch_fork = fork
+    pipe.order = order
+    if fork:
+        pipe.dispatch_fork = fork
     load_inputs(pipe, cfg, x, ids, rw)
     quantize_all_weights(pipe, cfg)
     pipe.run()

@@ -386,6 +386,53 @@ def test_gemv_from_the_routing_map_alone(mode, gemv_variant):
     np.testing.assert_array_equal(host_bf16_bits(out), host_bf16_bits(pipe.expert_out))
 
 
+IN_KERNEL_CASES = [
+    ("tiny", wl.config("tiny"), None),
+    ("decode_30b_a3b", wl.config("decode_30b_a3b"), None),
+    # more passes than CTAs: a CTA's range spans several passes (token lists)
+    ("many_passes", wl.small_config("many_passes", N=320, real=300, K=2048, E=256, top_k=8,
+                                    N_out=64, seed=21), None),
+    # one expert with many passes, through the decode variant
+    ("skewed", wl.small_config("skewed", N=400, real=391, K=1024, E=64, top_k=4, N_out=48,
+                               routing="zipf", zipf_s=1.6, seed=22), "mma"),
+    # three stages per block, 8-token passes, ragged row block
+    ("lines", wl.small_config("lines", N=40, real=37, K=2304, E=5, top_k=2, N_out=200), "mma"),
+]
+
+
+@pytest.mark.parametrize("name,cfg,variant", IN_KERNEL_CASES, ids=[c[0] for c in IN_KERNEL_CASES])
+def test_gemv_groups_the_map_in_kernel(name, cfg, variant, monkeypatch):
+    """Decode-sized W4A16 on the routing map alone: every CTA groups the map
+    itself (stable, as moe_create_indices defines it), and the result equals,
+    bit for bit, the same kernel handed the step-2 grouping -- with masked
+    rows, -1 and out-of-range ids in the map."""
+    if variant:
+        monkeypatch.setenv("MOE_GEMV_VARIANT", variant)
+    variant_id, in_kernel = moe.moe_grouped_gemv_plan(moe.MOE_W4A16, cfg.N, cfg.top_k, cfg.E,
+                                                      cfg.N_out, cfg.K)
+    assert variant_id == moe.MOE_GEMV_DECODE and in_kernel
+    pipe, x, ids = run_gemv_case(cfg, "w4a16")
+    m = pipe.routing_map.cpu().numpy()
+    rng = np.random.default_rng(9)
+    hit = rng.random(m.shape) < 0.03                  # ids that route nowhere
+    m[hit] = np.where(rng.random(hit.sum()) < 0.5, -1, cfg.E + 5)
+    pipe.routing_map.copy_(dev(m))
+    pipe.create_indices()
+    pipe.expert_out.view(torch.int16).fill_(SENTINEL)
+    pipe.gemv()                                       # on the grouping
+    torch.cuda.synchronize()
+    ref = host_bf16_bits(pipe.expert_out)
+    pipe.expert_out.view(torch.int16).fill_(SENTINEL)
+    pipe.gemv_on_map()                                # on the map alone
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(host_bf16_bits(pipe.expert_out), ref)
+    wq, sfw, gw = oracle_weights(cfg, range(cfg.E))
+    yref = oracle.grouped_gemv("w4a16", m, wq, sfw, gw, act_bf16=x)
+    routed = ~np.isnan(yref[..., 0])
+    assert np.all(ref[~routed] == SENTINEL)
+    assert_float_parity(host_bf16_f64(pipe.expert_out)[routed], yref[routed], what=name)
+
+
 def test_gemv_from_the_routing_map_follows_graph_replays():
     """The map is read on the device: a captured call follows new expert ids
     written between replays."""
