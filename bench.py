@@ -144,6 +144,9 @@ def algorithmic_bytes(cfg, mode: str, A: int, R: int, routed_tokens: int) -> dic
         act = routed_tokens * (K // 2 + K // 16)
     else:
         act = routed_tokens * K * 2
+    # the fused dispatch + quantisation reads every row once and writes both encodings
+    b["dispatch_quant"] = (N * K * 2 + R * stride + E * 4 + N * (K // 2 + K // 16)
+                           if mode == "w4a4" else 0)
     b["grouped_gemv"] = A * No * (K // 2 + K // 16) + act + R * No * 2 + A * 4
     b["combine"] = R * No * 2 + N * k * (4 + 8) + N * No * 2
     return b
@@ -313,7 +316,8 @@ def run_reference(args, rank, world):
 
 # ------------------------------------------------------------------ our arm
 # which entries of the byte model each launch of a step accounts for
-KERNEL_BYTES = {"mask+create_indices": ("mask", "create_indices")}
+KERNEL_BYTES = {"mask+create_indices": ("mask", "create_indices"),
+                "dispatch+quant_act": ("dispatch_quant",)}
 OTHER_WORKLOADS = ("tiny", "decode_large_expert", "prefill_index_stress", "gpt_oss_120b_w4a4")
 WORKLOAD_STEPS_CAP = 20    # timed steps per workload beyond the headline one
 
@@ -483,11 +487,12 @@ def measure_workload(cfg, mode, dev, steps, warmup, flush, peaks, weights, headl
     _, rows = replay_times(warmup + steps, kgraph,
                            after=lambda: [kev[i].elapsed_time(kev[i + 1]) for i in range(len(names))])
     per = {n: [row[i] for row in rows[warmup:]] for i, n in enumerate(names)}
-    bytes_ = algorithmic_bytes(cfg, mode, A, R, routed_tokens)
+    model = algorithmic_bytes(cfg, mode, A, R, routed_tokens)
+    bytes_ = {n: sum(model[k] for k in KERNEL_BYTES.get(n, (n,))) for n in names}
     kernels = {}
     for n in names:
         us = float(np.mean(per[n])) * 1e3
-        b = sum(bytes_[k] for k in KERNEL_BYTES.get(n, (n,)))
+        b = bytes_[n]
         rec = {"us": us, "algorithmic_bytes": b, "gbs": b / (us * 1e-6) / 1e9,
                "hbm_frac": b / (us * 1e-6) / 1e9 / hbm_peak}
         if n == "grouped_gemv":

@@ -211,6 +211,21 @@ MOE_API moe_status_t moe_dispatch_mxfp4(const void *input_tokens, int32_t N, int
                                 const uint32_t *expert_usage_stats, uint8_t *recv_buf,
                                 int64_t recv_capacity, uint32_t *recv_counts, cudaStream_t s);
 
+/* Steps 3 and 4a from one read of x (the W4A4 path needs both encodings */
+/* of the same rows: MAX ep.dispatch_async.mxfp4 execute(), and the       */
+/* FlashRT card's quantize_activations_nvfp4_bf16, whose                  */
+/* grouped_w4a4_gemv_from_bf16 path starts from the same bf16 rows).      */
+/* Writes exactly what moe_dispatch_mxfp4 (recv_buf, recv_counts) and     */
+/* moe_quantize_activations_nvfp4(x, N, K, act_global, xq, sfa) write,    */
+/* reading each token row once.  Arguments, limits and errors: as those   */
+/* two calls (xq uint8 [N, K/2], sfa uint8 [N, K/16]).                    */
+MOE_API moe_status_t moe_dispatch_mxfp4_quantize_nvfp4(
+    const void *input_tokens, int32_t N, int32_t K, int32_t top_k, int32_t E,
+    const uint32_t *restore_token_order, const uint32_t *expert_start_indices,
+    const int32_t *expert_ids, const uint32_t *expert_usage_stats, uint8_t *recv_buf,
+    int64_t recv_capacity, uint32_t *recv_counts, float act_global, uint8_t *xq, uint8_t *sfa,
+    cudaStream_t s);
+
 /* --------------------------------------------------------------------- */
 /* Step 4a -- FlashRT "grouped-moe-gemv" card, Available functions:       */
 /* quantize_activations_nvfp4_bf16.  For every 16-element block of       */

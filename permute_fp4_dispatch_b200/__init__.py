@@ -26,6 +26,7 @@ __all__ = [
     "moe_create_indices_static", "MOE_CREATE_INDICES_STATIC_SCRATCH",
     "moe_mask_and_create_indices",
     "moe_mxfp4_row_stride", "moe_dispatch_mxfp4", "moe_quantize_activations_nvfp4",
+    "moe_dispatch_mxfp4_quantize_nvfp4",
     "MOE_GEMV_DECODE", "MOE_GEMV_TENSOR_MEMORY", "MOE_GEMV_BLOCK_SCALED",
     "moe_quantize_weights_nvfp4", "moe_grouped_gemv_workspace_bytes", "moe_grouped_gemv_nvfp4",
     "moe_grouped_gemv_plan",
@@ -64,6 +65,8 @@ _SIGS = {
     "moe_mxfp4_row_stride": ([_I32], _SZ),
     "moe_dispatch_mxfp4": ([_P, _I32, _I32, _I32, _I32, _P, _P, _P, _P, _P, _I64, _P, _P], _I32),
     "moe_quantize_activations_nvfp4": ([_P, _I32, _I32, _F32, _P, _P, _P], _I32),
+    "moe_dispatch_mxfp4_quantize_nvfp4": ([_P, _I32, _I32, _I32, _I32, _P, _P, _P, _P, _P, _I64,
+                                           _P, _F32, _P, _P, _P], _I32),
     "moe_quantize_weights_nvfp4": ([_P, _I32, _I32, _I32, _P, _P, _P, _P], _I32),
     "moe_grouped_gemv_workspace_bytes": ([_I32, _I32, _I32], _SZ),
     "moe_grouped_gemv_nvfp4": ([_I32, _P, _P, _F32, _P, _I32, _I32, _P, _P, _P, _I32, _I32, _I32,
@@ -183,6 +186,18 @@ def moe_dispatch_mxfp4(input_tokens, N: int, K: int, top_k: int, E: int, restore
         _ptr(input_tokens), N, K, top_k, E, _ptr(restore_token_order),
         _ptr(expert_start_indices), _ptr(expert_ids), _ptr(expert_usage_stats), _ptr(recv_buf),
         recv_capacity, _ptr(recv_counts), _stream(stream)), "moe_dispatch_mxfp4")
+
+
+def moe_dispatch_mxfp4_quantize_nvfp4(input_tokens, N: int, K: int, top_k: int, E: int,
+                                      restore_token_order, expert_start_indices, expert_ids,
+                                      expert_usage_stats, recv_buf, recv_capacity: int,
+                                      recv_counts, act_global: float, xq, sfa, stream=None):
+    """moe_dispatch_mxfp4 and moe_quantize_activations_nvfp4 from one read of x."""
+    _check(library().moe_dispatch_mxfp4_quantize_nvfp4(
+        _ptr(input_tokens), N, K, top_k, E, _ptr(restore_token_order),
+        _ptr(expert_start_indices), _ptr(expert_ids), _ptr(expert_usage_stats), _ptr(recv_buf),
+        recv_capacity, _ptr(recv_counts), act_global, _ptr(xq), _ptr(sfa), _stream(stream)),
+        "moe_dispatch_mxfp4_quantize_nvfp4")
 
 
 def moe_quantize_activations_nvfp4(x, M: int, K: int, act_global: float, xq, sfa, stream=None):

@@ -188,9 +188,12 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
 }
 
 // Bounded wait: returns false (and raises MOE_DEVERR_WAIT_TIMEOUT) when the
-// phase has not completed within `limit_ns` nanoseconds.  A limit of 0 means
-// "no waiting at all": only a phase that has already completed passes (a
-// try_wait may suspend the thread for a while, so it is not used then).
+// phase has not completed within about `limit_ns` nanoseconds.  The limit is
+// kept in SM clock cycles (cheap to read, unlike the global timer), counted as
+// 2 cycles per nanosecond: at most the B200's top clock, so the wait is never
+// shorter than the limit.  A limit of 0 means "no waiting at all": only a
+// phase that has already completed passes (a try_wait may suspend the thread
+// for a while, so it is not used then).
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity,
                                                   uint64_t limit_ns) {
   if (limit_ns == 0) {
@@ -199,10 +202,11 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
     return false;
   }
   if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  while (true) {
+  const long long t0 = clock64();
+  const long long limit = (long long)(limit_ns * 2u);
+  for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (globaltimer_ns() - t0 > limit_ns) {
+    if ((i & 15u) == 0u && clock64() - t0 > limit) {
       raise_device_error(MOE_DEVERR_WAIT_TIMEOUT);
       return false;
     }

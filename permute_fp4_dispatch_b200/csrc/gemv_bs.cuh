@@ -285,8 +285,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       // row's 16 scale bytes of the stage (8 rows per instruction).  Rows the
       // MMA result does not use -- tokens past the pass, weight rows past N --
       // are not copied: D row i depends only on A row i, column j only on B row j.
-      const int bj = t & 7, bt0 = t >> 3;        // B: chunk bj of token bt0 + 16 * it
-      const int skk = t & 3, sr0 = t >> 2;       // scales: word skk of row sr0 + 32 * it
+      const int bj = t & 7, bt0 = t >> 3;        // B: chunk bj of token bt0 + 16 * i
+      const int skk = t & 3, sr0 = t >> 2;       // scales: word skk of row sr0 + 32 * i
+      // this thread's source rows for the whole unit (token rows of x, rows of
+      // the weight scales); a row the unit does not use gets offset -1
+      int64_t brow[kTS / 16], arow[4], srow[4];
+#pragma unroll
+      for (int i = 0; i < kTS / 16; ++i) {
+        const int tok = bt0 + 16 * i;
+        brow[i] = tok < r.ntok ? (int64_t)(pairs[tok] / (uint32_t)p.top_k) * xrow : -1;
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int row = sr0 + 32 * i;
+        arow[i] = r.n0 + row < N ? ((int64_t)r.e * N + r.n0 + row) * sfrow : -1;
+        srow[i] = row < r.ntok ? (int64_t)(pairs[row] / (uint32_t)p.top_k) * sfrow : -1;
+      }
       for (int c = 0; c < nst; ++c, ++it) {
         const int s = (int)(it % kStages);
         wait(&empty[s], ((it / kStages) & 1u) ^ 1u);
@@ -298,22 +312,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int i = 0; i < kTS / 16; ++i) {
             const int tok = bt0 + 16 * i;
-            if (tok < r.ntok && bchunk) {
-              const uint8_t *src = xq + (int64_t)(pairs[tok] / (uint32_t)p.top_k) * xrow + kb0 + 16 * bj;
-              cp_async16_zfill(bt + tok * 128 + ((bj ^ (tok & 7)) << 4), src, 16u);
-            }
+            if (brow[i] >= 0 && bchunk)
+              cp_async16_zfill(bt + tok * 128 + ((bj ^ (tok & 7)) << 4),
+                               xq + brow[i] + kb0 + 16 * bj, 16u);
           }
           const int kc = c * (kKC / 16) + 4 * skk;  // first scale byte of MMA skk of the stage
           if (kc + 4 <= sfrow) {
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-              const int row = sr0 + 32 * i;
-              const int off = skk * kSFStep + (row & 31) * 16 + (row >> 5) * 4;
-              if (r.n0 + row < N)
-                cp_async4_zfill(sfa_s + off, p.sfw + ((int64_t)r.e * N + r.n0 + row) * sfrow + kc, 4u);
-              if (row < r.ntok)
-                cp_async4_zfill(sfb_s + off,
-                                p.sfa + (int64_t)(pairs[row] / (uint32_t)p.top_k) * sfrow + kc, 4u);
+              const int off = skk * kSFStep + sr0 * 16 + i * 4;  // row sr0 + 32 i of the layout
+              if (arow[i] >= 0) cp_async4_zfill(sfa_s + off, p.sfw + arow[i] + kc, 4u);
+              if (srow[i] >= 0) cp_async4_zfill(sfb_s + off, p.sfa + srow[i] + kc, 4u);
             }
           }
         }

@@ -13,26 +13,37 @@
 //     at round boundaries; rounds of up to 16 blocks of one (expert, pass),
 //     warp w owns block w of every round.  The CTA computes its range once,
 //     after each CTA has pulled its slice of the bf16 activations into L2
-//     while waiting for the routing kernel (programmatic launch).
-//   * Every warp runs its own one-stage pipeline, with no producer warp and
-//     no cross-warp waits inside a pass; sixteen warps (four per scheduler)
-//     hide each other's load and dependency latencies.  A stage is 16 rows x
-//     1024 codes:
-//     one 4-D TMA box (16 rows x 4 lines of 128 bytes, 512 contiguous bytes
-//     per row, 128-byte swizzle, L2 evict-first) plus one 3-D box of the
-//     stage's 16 x 64 E4M3 scale bytes, both issued by lane 0 and completing
-//     on the stage's mbarrier.  The TMA engine's cost grows with
-//     the number of contiguous runs it fetches; 512-byte runs stream at the
-//     rate of plain bulk copies where 128-byte runs do not.
+//     while waiting for the previous kernel (programmatic launch).
+//   * Handed the routing map without the step-2 grouping (at most 4096
+//     slots, 512 experts), every CTA groups the map itself: per-expert counts
+//     (shared-memory histogram), the active experts' CSR offsets (block scan),
+//     and the token lists of the passes in its own range (a stable block-wide
+//     compaction per expert), so no grouping kernel precedes it.
+//   * Each pair of warps shares a one-stage pipeline, with no producer warp
+//     and no waits beyond the pair inside a pass; sixteen warps (four per
+//     scheduler) hide each other's load and dependency latencies.  A stage
+//     is the pair's two 16-row blocks x 1024 codes: one 4-D TMA box (32 rows
+//     x 4 lines of 128 bytes, 512 contiguous bytes per row, 128-byte
+//     swizzle, L2 evict-first) plus one 3-D box of the stage's 32 x 64 E4M3
+//     scale bytes, both issued by the even warp's lane 0 and completing on
+//     the stage's mbarrier; each warp then releases the stage on a second
+//     barrier, and the even warp refills it once both have.  The TMA
+//     engine's throughput grows with the size of its boxes: 16 KB boxes
+//     stream about 1.6x faster than 8 KB ones at the same bytes in flight.
 //   * Lane (g, t) owns line t of rows g and g + 8.  A line index in the box is
 //     4 * row + line, so the swizzle key is (row & 1) * 4 + line and the eight
 //     lanes of one shared-memory phase (rows g, g + 1) hit eight distinct
 //     16-byte bank groups.
 //   * When a CTA starts a new (expert, pass), its 16 warps convert that
 //     pass's activation rows once, for the whole K, into an fp16 tile laid
-//     out in mma fragment order; every round of the pass reuses it.  W4A16: plain
-//     bf16 -> fp16 (exact for 2^-14 <= |x| <= 65504, MOE_DEVERR_ACT_RANGE
-//     beyond); W4A4: E2M1 x E4M3 products, exact in fp16.
+//     out in mma fragment order; every round of the pass reuses it.  W4A16:
+//     each token is scaled by a power of two of its own so that its largest
+//     element lands in [2^14, 2^15), then converted to fp16 -- exact for every
+//     element within 2^29 of the token's maximum, whatever the token's
+//     magnitude (bf16's whole range), and bit-identical to no scaling when the
+//     token already fits fp16 (fp32 accumulation rounds alike at any power-of-
+//     two scale); the epilogue multiplies each token column back.  W4A4:
+//     E2M1 x E4M3 products, exact in fp16.
 //   * Each lane dequantises its codes in registers (hardware E2M1 -> f16x2
 //     converter, times the block's E4M3 scale: exact in fp16) and issues
 //     m16n8k16 MMAs (fp32 accumulation, two independent chains per 8-token
@@ -52,11 +63,12 @@ constexpr int kCW = 16;                      // warps, one 16-row block each per
 constexpr int kThreads = kCW * 32;
 constexpr int kLines = 4;                    // 128-byte lines (256 codes) per row per stage
 constexpr int kKS = kLines * 256;            // codes per row per stage
-constexpr int kSlots = 1;                    // pipeline stages per warp
+constexpr int kPairs = kCW / 2;              // warp pairs; a pair shares one 32-row stage
 constexpr int kRowW = kLines * 128;          // bytes of codes per row per stage
 constexpr int kRowSF = kLines * 16;          // scale bytes per row per stage
-constexpr int kStageW = 16 * kRowW;          // 8 KB
-constexpr int kStageSF = 16 * kRowSF;        // 1 KB
+constexpr int kStageRows = 32;               // rows per stage: the pair's two blocks
+constexpr int kStageW = kStageRows * kRowW;  // 16 KB
+constexpr int kStageSF = kStageRows * kRowSF;  // 2 KB
 constexpr int kMaxTS = 16;                   // tokens per pass at most (2 groups of 8)
 constexpr int kNG = kMaxTS / 8;
 constexpr int kGroupStageBytes = 8 * kKS * 2;  // fp16 tile of one 8-token group x one stage
@@ -68,8 +80,8 @@ constexpr uint64_t kActPrefetchMax = 8u << 20;     // activations prefetched int
 constexpr int kSetupTasks = kActBytes / 16 / kThreads;
 
 constexpr size_t kOffW = 0;
-constexpr size_t kOffSF = kOffW + (size_t)kCW * kSlots * kStageW;
-constexpr size_t kOffAct = kOffSF + (size_t)kCW * kSlots * kStageSF;
+constexpr size_t kOffSF = kOffW + (size_t)kPairs * kStageW;
+constexpr size_t kOffAct = kOffSF + (size_t)kPairs * kStageSF;
 constexpr size_t kOffStaging = kOffAct + kActBytes;
 constexpr int kMaxActive = 512;              // active experts this variant takes
 constexpr size_t kOffPrefix = kOffStaging + kStagingBytes;
@@ -86,8 +98,9 @@ constexpr int kFusedPer = kFusedSlots / kThreads;  // slots per thread
 constexpr int kMaxCtaPasses = 16;
 constexpr size_t kOffPasses = kOffPair + kMaxTS * 4;                 // [kMaxCtaPasses][kMaxTS]
 constexpr size_t kOffPassMeta = kOffPasses + (size_t)kMaxCtaPasses * kMaxTS * 4;  // [3][kMaxCtaPasses]
-constexpr size_t kOffBar = kOffPassMeta + (size_t)3 * kMaxCtaPasses * 4 + 8;
-constexpr size_t kOffMisc = kOffBar + (size_t)kCW * kSlots * 8;
+constexpr size_t kOffTokMax = kOffPassMeta + (size_t)3 * kMaxCtaPasses * 4 + 8;  // [2][kMaxTS]
+constexpr size_t kOffBar = kOffTokMax + (size_t)2 * kMaxTS * 4;
+constexpr size_t kOffMisc = kOffBar + (size_t)2 * kPairs * 8;  // full[kPairs], empty[kPairs]
 constexpr size_t kSmemBytes = kOffMisc + 16 + 1024;
 static_assert(kStageW % 1024 == 0, "stages must keep the 1024-byte swizzle alignment");
 static_assert(kOffBar % 8 == 0, "mbarrier alignment");
@@ -109,6 +122,18 @@ __host__ __device__ constexpr int tokens_per_pass(int K) {
 __device__ __forceinline__ int act_index(int c, int ng, int G, int m, int lane) {
   return (((c * ng + G) * 32 + m) << 5) + lane;
 }
+
+// W4A16 tokens enter the tensor cores as fp16 scaled by a power of two of
+// their own: s = floor(log2(amax)) - 14 (clamped to [-126, 127]), so the
+// token's largest element lands in [2^14, 2^15) and every bf16 value of the
+// token within 2^29 of it is exact in fp16.  amax_bits are the fp32 bits of
+// the token's largest magnitude.
+__device__ __forceinline__ int token_shift(uint32_t amax_bits) {
+  if (amax_bits == 0u) return 0;
+  int s = (int)((amax_bits >> 23) & 0xFFu) - 127 - 14;
+  return s < -126 ? -126 : (s > 127 ? 127 : s);
+}
+__device__ __forceinline__ float pow2f(int s) { return __uint_as_float((uint32_t)(s + 127) << 23); }
 
 __device__ __forceinline__ uint32_t word_of(const uint4 &v, int i) {
   return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
@@ -230,9 +255,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   // set-up that reads no input runs before the wait for the previous grid
   if (threadIdx.x == 0) {
     // one arrival with the byte count of the stage's two TMA boxes
-    for (int i = 0; i < kCW * kSlots; ++i) mbar_init(&full[i], 1u);
+    for (int i = 0; i < kPairs; ++i) {
+      mbar_init(&full[i], 1u);              // the leader's expect-tx arrival
+      mbar_init(&full[kPairs + i], 2u);     // "empty": both warps of the pair are done
+    }
     *abort_flag = 0;
     fence_mbar_init();
+  }
+  if (threadIdx.x < 2 * kMaxTS) {
+    reinterpret_cast<uint32_t *>(smem + kOffTokMax)[threadIdx.x] = 0u;
   }
   if (lane == 0) {
     prefetch_tmap(&tmap_w);
@@ -363,12 +394,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
   }
   int pass_idx = -1;  // index of the current pass in s_passes
-  uint8_t *wring = smem + kOffW + (size_t)warp * kSlots * kStageW;
-  uint8_t *sring = smem + kOffSF + (size_t)warp * kSlots * kStageSF;
-  uint64_t *wfull = full + warp * kSlots;
+  const int pair = warp >> 1, half = warp & 1;
+  const bool leader = half == 0;  // the pair's even warp issues the pair's copies
+  uint8_t *pw = smem + kOffW + (size_t)pair * kStageW;
+  uint8_t *ps = smem + kOffSF + (size_t)pair * kStageSF;
+  uint64_t *pfull = full + pair;
+  uint64_t *pempty = full + kPairs + pair;
   const uint64_t policy = l2_evict_first_policy();
 
-  // ---- producer side of this warp's pipeline: the next (round, stage) of its blocks
+  // ---- producer side of the pair's pipeline (leader warp): the next (round, stage)
+  // in which the pair holds a block
   RoundWalk piter;
   piter.init(meta, A, RB, u_begin, u_end);
   Round pr;
@@ -378,7 +413,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     pvalid = false;
     pc = 0;
     while (piter.next(meta, RB, (uint32_t)ts, pr))
-      if (warp < pr.nblk) {
+      if (2 * pair < pr.nblk) {
         pvalid = true;
         break;
       }
@@ -387,18 +422,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t produced = 0;
   auto produce = [&]() {
     // lane 0's view of the abort flag decides for the whole warp
-    if (!pvalid || __shfl_sync(0xFFFFFFFFu, *abort_flag, 0)) return;
-    const int slot = (int)(produced % kSlots);
-    uint8_t *sw = wring + slot * kStageW;
-    uint8_t *ssf = sring + slot * kStageSF;
-    uint64_t *bar = &wfull[slot];
-    const int n0 = pr.n0 + 16 * warp;
+    if (!leader || !pvalid || __shfl_sync(0xFFFFFFFFu, *abort_flag, 0)) return;
+    // the stage is refilled once both warps of the pair have released its previous contents
+    if (produced > 0 && !mbar_wait_bounded(pempty, (produced - 1) & 1u, p.wait_limit_ns))
+      *abort_flag = 1;
+    if (__shfl_sync(0xFFFFFFFFu, *abort_flag, 0)) return;
+    const int n0 = pr.n0 + 32 * pair;
     if (lane == 0) {
-      mbar_arrive_expect_tx(bar, (uint32_t)(kStageW + kStageSF));
-      tma_load_4d(sw, &tmap_w, 0, pc * kLines, n0, pr.e, bar, policy);
-      // scales: 16 rows x 4 words (one 16-byte group per line), rows beyond N and
+      mbar_arrive_expect_tx(pfull, (uint32_t)(kStageW + kStageSF));
+      tma_load_4d(pw, &tmap_w, 0, pc * kLines, n0, pr.e, pfull, policy);
+      // scales: 32 rows x 4 words (one 16-byte group per line), rows beyond N and
       // lines beyond K read as zero
-      tma_load_3d(ssf, &tmap_sf, pc * kLines * 4, n0, pr.e, bar, policy);
+      tma_load_3d(ps, &tmap_sf, pc * kLines * 4, n0, pr.e, pfull, policy);
     }
     ++produced;
     if (++pc == nst) next_own_round();
@@ -464,14 +499,40 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (kk += kThreads; kk >= per_tok; kk -= per_tok) ++tau;
       }
+      // W4A16: every token's largest magnitude (a warp's lanes share a token per
+      // task, so one atomic per warp and task), into this pass's buffer
+      uint32_t *tokmax = reinterpret_cast<uint32_t *>(smem + kOffTokMax) + (pass_idx & 1) * kMaxTS;
+      if (MODE == MOE_W4A16) {
+        int tm = tau0;
+        int km = kk0;
+#pragma unroll
+        for (int b = 0; b < kSetupTasks; ++b) {
+          const int task = b * kThreads + (int)threadIdx.x;
+          const int tk = tm;
+          for (km += kThreads; km >= per_tok; km -= per_tok) ++tm;
+          if (task - (int)lane >= ntask) continue;  // warp-uniform: the whole warp is past the tasks
+          uint32_t mx = 0u;
+          if (task < ntask) {
+            const uint32_t w4[4] = {v[b].x, v[b].y, v[b].z, v[b].w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              mx = max(mx, max((w4[i] << 16) & 0x7FFF0000u, w4[i] & 0x7FFF0000u));
+          }
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+          if (lane == 0 && mx) atomicMax(&tokmax[tk], mx);
+        }
+      }
       if (!primed) {
-        for (int st = 0; st < kSlots; ++st) produce();
+        produce();
         primed = true;
       }
       if (pass_key != 0xFFFFFFFFu) named_bar_sync(1, kThreads);  // previous tile no longer read
+      // the other maxima buffer served the previous pass, which is done: clear it for the next
+      if (MODE == MOE_W4A16 && (int)threadIdx.x < kMaxTS)
+        reinterpret_cast<uint32_t *>(smem + kOffTokMax)[((pass_idx + 1) & 1) * kMaxTS + threadIdx.x] = 0u;
       ng = (r.ntok + 7) / 8;
       if ((int)threadIdx.x < r.ntok) s_pair[threadIdx.x] = my_pair;
-      unsigned range_bad = 0;
       tau = tau0;
       kk = kk0;
 #pragma unroll
@@ -483,13 +544,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint4 hv = make_uint4(0u, 0u, 0u, 0u);
         if (k < K) {
           if (MODE == MOE_W4A16) {
+            // scaled by the token's power of two (exact), then fp16 (exact in range)
+            const float down = pow2f(-token_shift(tokmax[tk]));
             float f[8];
             f[0] = bf16_lo(v[b].x); f[1] = bf16_hi(v[b].x);
             f[2] = bf16_lo(v[b].y); f[3] = bf16_hi(v[b].y);
             f[4] = bf16_lo(v[b].z); f[5] = bf16_hi(v[b].z);
             f[6] = bf16_lo(v[b].w); f[7] = bf16_hi(v[b].w);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) range_bad |= (fabsf(f[e]) > 65504.0f) ? 1u : 0u;
+            for (int e = 0; e < 8; ++e) f[e] = __fmul_rn(f[e], down);
             hv.x = pack_f16x2(f[0], f[1]);
             hv.y = pack_f16x2(f[2], f[3]);
             hv.z = pack_f16x2(f[4], f[5]);
@@ -508,12 +571,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int c = k / kKS, kc = k % kKS, lt = kc / 256, m = (kc % 256) / 8;
         act[act_index(c, ng, tk / 8, m, (tk & 7) * 4 + lt)] = hv;
       }
-      if (MODE == MOE_W4A16 && range_bad) raise_device_error(MOE_DEVERR_ACT_RANGE);
       named_bar_sync(1, kThreads);
       pass_key = r.tok0;
     }
 
-    if (warp >= r.nblk) continue;
+    if (2 * pair >= r.nblk) continue;  // the pair holds no block of this round
+    const bool own = warp < r.nblk;     // this warp's block (the odd warp may have none)
     const float gw = p.w_global ? __ldg(p.w_global + r.e) : 1.0f;  // used by the epilogue
     float acc0[kNG][4], acc1[kNG][4];
 #pragma unroll
@@ -522,13 +585,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = 0; i < 4; ++i) acc0[G][i] = acc1[G][i] = 0.f;
 
     for (int c = 0; c < nst; ++c) {
-      const int slot = (int)(consumed % kSlots);
-      if (!*abort_flag &&
-          !mbar_wait_bounded(&wfull[slot], (consumed / kSlots) & 1u, p.wait_limit_ns))
+      if (!*abort_flag && !mbar_wait_bounded(pfull, consumed & 1u, p.wait_limit_ns))
         *abort_flag = 1;
-      if (!*abort_flag) {
-        const uint8_t *sw = wring + slot * kStageW;
-        const uint8_t *ssf = sring + slot * kStageSF;
+      if (!*abort_flag && own) {
+        // this warp's 16 rows of the pair's stage
+        const uint8_t *sw = pw + (size_t)half * 16 * kRowW;
+        const uint8_t *ssf = ps + (size_t)half * 16 * kRowSF;
         const bool line_ok = c * kLines + t < lines_total;
         const uint4 *act_c = act + act_index(c, ng, 0, 0, 0);
         if (ng == 1)
@@ -537,19 +599,31 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_stage<2>(sw, ssf, act_c, g, t, lane, line_ok, acc0, acc1);
       }
       ++consumed;
-      __syncwarp();  // every lane is done with the slot before it is refilled
+      __syncwarp();  // every lane is done with the stage
+      if (lane == 0) mbar_arrive(pempty);
       produce();
     }
 
     // ---- block epilogue: scale, round to bf16, transpose, 16-byte stores
-    if (!*abort_flag) {
+    if (!*abort_flag && own) {
       const float f = __fmul_rn(gw, p.g_a);
       uint16_t *st = staging + warp * (kMaxTS * 16);
-      auto y = [&](int G, int i) { return __fmul_rn(acc0[G][i] + acc1[G][i], f); };
+      const uint32_t *tokmax = reinterpret_cast<const uint32_t *>(smem + kOffTokMax) +
+                               (pass_idx & 1) * kMaxTS;
+      float up0 = 1.0f, up1 = 1.0f;  // the power of two of this lane's two token columns
+      // g_w * g_a first, the token's power of two last: the product then never
+      // overflows early, and it rounds exactly as the unscaled one would
+      auto y = [&](int G, int i) {
+        return __fmul_rn(__fmul_rn(acc0[G][i] + acc1[G][i], f), (i & 1) ? up1 : up0);
+      };
 #pragma unroll
       for (int G = 0; G < kNG; ++G) {
         if (G < ng) {
           const int c0 = G * 8 + 2 * t;
+          if (MODE == MOE_W4A16) {
+            up0 = pow2f(token_shift(tokmax[c0]));
+            up1 = pow2f(token_shift(tokmax[c0 + 1]));
+          }
           const uint32_t lo = pack_bf16x2(y(G, 0), y(G, 1));
           const uint32_t hi = pack_bf16x2(y(G, 2), y(G, 3));
           st[c0 * 16 + g] = (uint16_t)(lo & 0xFFFFu);
@@ -573,15 +647,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
-  // After a timed-out wait, let this warp's copies still in flight land
+  // After a timed-out wait, let the pair's copies still in flight land
   // before the CTA exits (bounded again).
-  if (*abort_flag && lane == 0) {
-    for (int s = 0; s < kSlots; ++s) {
-      const uint32_t uses =
-          produced > (uint32_t)s ? (produced - (uint32_t)s + kSlots - 1) / kSlots : 0u;
-      if (uses) mbar_wait_bounded(&wfull[s], (uses - 1) & 1u, kDrainLimitNs);
-    }
-  }
+  if (*abort_flag && leader && lane == 0 && produced > 0)
+    mbar_wait_bounded(pfull, (produced - 1) & 1u, kDrainLimitNs);
 }
 
 }  // namespace mma

@@ -17,6 +17,7 @@
 #include "common.cuh"
 #include "create_indices.cuh"
 #include "dispatch_mxfp4.cuh"
+#include "dispatch_quant.cuh"
 #include "gemv_bs.cuh"
 #include "gemv_mma.cuh"
 #include "gemv_tc.cuh"
@@ -143,16 +144,15 @@ bool encode_u8_3d(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// 4-D uint32 map over the codes of [E][N][K/2] seen as [E][N][K/256 lines]
-// [32 words of a 128-byte line]; box = 16 rows x `lines` lines, 128-byte
-// swizzle.  Needs K % 256 == 0.
+// 4-D uint32 map over the codes of [E][N][K/256 lines][32 words of a 128-byte
+// line]; box = `rows` rows x `lines` lines, 128-byte swizzle.  Needs K % 256 == 0.
 bool encode_lines_4d(CUtensorMap *m, const void *base, uint64_t K, uint64_t N, uint64_t E,
-                     uint32_t lines) {
+                     uint32_t lines, uint32_t rows) {
   auto fn = tensor_map_encoder();
   if (!fn) return false;
   const cuuint64_t dims[4] = {32, K / 256, N, E};
   const cuuint64_t strides[3] = {128, K / 2, (K / 2) * N};
-  const cuuint32_t box[4] = {32, lines, 16, 1};
+  const cuuint32_t box[4] = {32, lines, rows, 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, const_cast<void *>(base), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -160,14 +160,14 @@ bool encode_lines_4d(CUtensorMap *m, const void *base, uint64_t K, uint64_t N, u
 }
 
 // 3-D uint32 map over the scales [E][N][K/16 bytes] seen as [E][N][K/64 words];
-// box = 16 rows x `words` words, no swizzle.  Needs K % 256 == 0 (16-byte rows).
+// box = `rows` rows x `words` words, no swizzle.  Needs K % 256 == 0 (16-byte rows).
 bool encode_scale_words_3d(CUtensorMap *m, const void *base, uint64_t K, uint64_t N, uint64_t E,
-                           uint32_t words) {
+                           uint32_t words, uint32_t rows) {
   auto fn = tensor_map_encoder();
   if (!fn) return false;
   const cuuint64_t dims[3] = {K / 64, N, E};
   const cuuint64_t strides[2] = {K / 16, (K / 16) * N};
-  const cuuint32_t box[3] = {words, 16, 1};
+  const cuuint32_t box[3] = {words, rows, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<void *>(base), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -220,10 +220,12 @@ bool library_maps(const uint8_t *w, const uint8_t *sfw, int E, int N, int K, Lib
                                 CU_TENSOR_MAP_SWIZZLE_NONE))
     return false;
   if (m.sf_tma && !encode_lines_4d(&m.tlines, w, (uint64_t)K, (uint64_t)N, (uint64_t)E,
-                                   (uint32_t)moe::gemv::mma::kLines))
+                                   (uint32_t)moe::gemv::mma::kLines,
+                                   (uint32_t)moe::gemv::mma::kStageRows))
     return false;
   if (m.sf_tma && !encode_scale_words_3d(&m.tsf_lines, sfw, (uint64_t)K, (uint64_t)N, (uint64_t)E,
-                                         (uint32_t)moe::gemv::mma::kLines * 4))
+                                         (uint32_t)moe::gemv::mma::kLines * 4,
+                                         (uint32_t)moe::gemv::mma::kStageRows))
     return false;
   g_maps[g_maps_next] = m;
   g_maps_next = (g_maps_next + 1) % kMapCache;
@@ -409,6 +411,49 @@ moe_status_t moe_dispatch_mxfp4(const void *input_tokens, int32_t N, int32_t K, 
                     static_cast<const uint16_t *>(input_tokens), N, K, top_k, E,
                     restore_token_order, expert_start_indices, expert_ids, expert_usage_stats,
                     recv_buf, recv_capacity, (int32_t)moe_mxfp4_row_stride(K), recv_counts);
+}
+
+moe_status_t moe_dispatch_mxfp4_quantize_nvfp4(
+    const void *input_tokens, int32_t N, int32_t K, int32_t top_k, int32_t E,
+    const uint32_t *restore_token_order, const uint32_t *expert_start_indices,
+    const int32_t *expert_ids, const uint32_t *expert_usage_stats, uint8_t *recv_buf,
+    int64_t recv_capacity, uint32_t *recv_counts, float act_global, uint8_t *xq, uint8_t *sfa,
+    cudaStream_t s) {
+  if (N < 0 || K <= 0 || K % 32 != 0 || top_k < 1 || E < 1 || E > 1024 || top_k > E ||
+      recv_capacity < 0 || !(act_global > 0.0f))
+    return MOE_ERR_INVALID_ARG;
+  if (!expert_start_indices || !expert_ids || !expert_usage_stats || !recv_counts)
+    return MOE_ERR_INVALID_ARG;
+  if (N > 0 && (!input_tokens || !restore_token_order || !xq || !sfa)) return MOE_ERR_INVALID_ARG;
+  if (recv_capacity > 0 && !recv_buf) return MOE_ERR_INVALID_ARG;
+  if (!aligned(input_tokens, 16) || !aligned(recv_buf, 16) || !aligned(recv_counts, 4) ||
+      !aligned(xq, 4))
+    return MOE_ERR_INVALID_ARG;
+  int sms = 0;
+  moe_status_t st = check_device(&sms);
+  if (st != MOE_OK) return st;
+  // the dispatch's launch shape: segments of 256 columns per warp task, the
+  // largest of 8, 4, 2, 1 that still gives every SM about 8 warps
+  const int wpb = moe::disp::kWarpsPerBlock;
+  const int64_t segs = (K + 255) / 256;
+  int seg = 8;
+  while (seg > 1 && (int64_t)N * ((segs + seg - 1) / seg) < (int64_t)sms * 8) seg /= 2;
+  const int64_t groups = (segs + seg - 1) / seg;
+  int64_t blocks = ((int64_t)N * groups + wpb - 1) / wpb;
+  if (blocks < 1) blocks = 1;
+  if (blocks > (int64_t)sms * 16) blocks = (int64_t)sms * 16;
+  void (*kern)(const uint16_t *, int32_t, int32_t, int32_t, int32_t, const uint32_t *,
+               const uint32_t *, const int32_t *, const uint32_t *, uint8_t *, int64_t, int32_t,
+               uint32_t *, float, uint8_t *, uint8_t *) =
+      seg == 8   ? moe::dq::dispatch_quant_kernel<8>
+      : seg == 4 ? moe::dq::dispatch_quant_kernel<4>
+      : seg == 2 ? moe::dq::dispatch_quant_kernel<2>
+                 : moe::dq::dispatch_quant_kernel<1>;
+  return launch_pdl(kern, dim3((unsigned)blocks), dim3(wpb * 32), 0, s,
+                    static_cast<const uint16_t *>(input_tokens), N, K, top_k, E,
+                    restore_token_order, expert_start_indices, expert_ids, expert_usage_stats,
+                    recv_buf, recv_capacity, (int32_t)moe_mxfp4_row_stride(K), recv_counts,
+                    act_global, xq, sfa);
 }
 
 // ------------------------------------------------------------------ step 4a

@@ -19,7 +19,8 @@ from . import (MOE_EPI_IDENTITY, MOE_EPI_NONE, MOE_EPI_SCALE, MOE_W4A4, MOE_W4A1
                moe_combine, moe_create_indices, moe_create_indices_workspace_bytes,
                moe_mask_and_create_indices, moe_grouped_gemv_plan,
                moe_grouped_gemv_workspace_bytes,
-               moe_dispatch_mxfp4, moe_grouped_gemv_nvfp4, moe_mask_padding,
+               moe_dispatch_mxfp4, moe_dispatch_mxfp4_quantize_nvfp4, moe_grouped_gemv_nvfp4,
+               moe_mask_padding,
                moe_mxfp4_row_stride, moe_quantize_activations_nvfp4, moe_quantize_weights_nvfp4)
 
 EPILOGUES = {"none": MOE_EPI_NONE, "identity": MOE_EPI_IDENTITY, "scale": MOE_EPI_SCALE}
@@ -116,6 +117,9 @@ class RoutingPipeline:
         # map itself (decode-sized W4A16), so grouping is off its critical path.
         _, in_kernel = moe_grouped_gemv_plan(self.gemv_mode, N, top_k, E, N_out, K)
         self.order = "gemv_groups" if in_kernel else "routing_first"
+        # W4A4 in the "routing_first" order: the MXFP4 dispatch and the NVFP4
+        # activation quantisation as one kernel (one read of x) before the GEMV
+        self.fuse_dispatch_quant = self.gemv_mode == MOE_W4A4 and dispatch
         # step 5
         self.output = torch.empty((N, N_out), dtype=torch.bfloat16, device=dev)
         # timing events go on a side stream, so no event sits between two kernels
@@ -167,6 +171,14 @@ class RoutingPipeline:
         moe_dispatch_mxfp4(self.x, self.N, self.K, self.top_k, self.E, self.restore_token_order,
                            self.expert_start_indices, self.expert_ids, self.expert_usage_stats,
                            self.recv_buf, self.recv_capacity, self.recv_counts, stream)
+
+    def dispatch_quantize(self, stream=None):
+        """The MXFP4 dispatch and the NVFP4 activation quantisation from one
+        read of x (W4A4)."""
+        moe_dispatch_mxfp4_quantize_nvfp4(
+            self.x, self.N, self.K, self.top_k, self.E, self.restore_token_order,
+            self.expert_start_indices, self.expert_ids, self.expert_usage_stats, self.recv_buf,
+            self.recv_capacity, self.recv_counts, self.act_global, self.xq, self.sfa, stream)
 
     def quantize_activations(self, stream=None):
         moe_quantize_activations_nvfp4(self.x, self.N, self.K, self.act_global, self.xq,
@@ -245,6 +257,17 @@ class RoutingPipeline:
 
     def _run_routing_first(self, main, gemv_events, side_stream, x_ready):
         self.mask_and_create_indices(main)
+        if self.fuse_dispatch_quant:
+            if x_ready is not None:
+                main.wait_event(x_ready)
+            self.dispatch_quantize(main)
+            if gemv_events is not None:
+                self._mark(main, gemv_events[0])
+            self.gemv(main)
+            if gemv_events is not None:
+                self._mark(main, gemv_events[1])
+            self.combine(main)
+            return
         forked = self.dispatch and side_stream is not None
         early = forked and self.dispatch_fork == "routing"
         if early:
@@ -295,10 +318,13 @@ class RoutingPipeline:
             steps = [("mask", self.mask), ("create_indices", self.create_indices)]
         else:
             steps = [("mask+create_indices", self.mask_and_create_indices)]
-        if self.dispatch:
-            steps.append(("dispatch_mxfp4", self.dispatch_mxfp4))
-        if self.gemv_mode == MOE_W4A4:
-            steps.append(("quant_act_nvfp4", self.quantize_activations))
+        if self.order == "routing_first" and self.fuse_dispatch_quant:
+            steps.append(("dispatch+quant_act", self.dispatch_quantize))
+        else:
+            if self.dispatch:
+                steps.append(("dispatch_mxfp4", self.dispatch_mxfp4))
+            if self.gemv_mode == MOE_W4A4:
+                steps.append(("quant_act_nvfp4", self.quantize_activations))
         gemv = self.gemv_on_map if self.order == "gemv_groups" else self.gemv
         steps.append(("grouped_gemv", gemv))
         steps.append(("combine", self.combine))
@@ -312,6 +338,9 @@ class RoutingPipeline:
             n = 1 + ci + 1                       # mask, create_indices, GEMV (groups in-kernel)
         else:
             n = (1 if self.S <= 1024 else 1 + ci) + 1
-        n += 1 if self.dispatch else 0
-        n += 1 if self.gemv_mode == MOE_W4A4 else 0
+        if self.order == "routing_first" and self.fuse_dispatch_quant:
+            n += 1
+        else:
+            n += 1 if self.dispatch else 0
+            n += 1 if self.gemv_mode == MOE_W4A4 else 0
         return n + 1                             # combine

@@ -257,6 +257,40 @@ def test_dispatch_capacity_overflow_is_reported():
     np.testing.assert_array_equal(pipe.recv_buf.cpu().numpy(), ref_recv[:10])
 
 
+@pytest.mark.parametrize("cfg", [
+    wl.config("tiny"),
+    wl.small_config("dq_large_k", N=300, real=290, K=7168, E=16, top_k=8),
+    wl.small_config("dq_ragged", N=64, real=50, K=2880, E=12, top_k=4, outlier_frac=0.01,
+                    outlier_mult=20.0),
+    wl.small_config("dq_k32", N=33, real=33, K=96, E=5, top_k=2),
+])
+def test_dispatch_quantize_fused_equals_separate(cfg):
+    """Steps 3 and 4a from one read of x give byte for byte what the two
+    separate calls give (MXFP4 rows and counts, NVFP4 codes and scales)."""
+    x = wl.activations_bf16(cfg)
+    pipe = RoutingPipeline(cfg.N, cfg.K, cfg.E, cfg.top_k, 64, mode="w4a4", act_global=0.375)
+    load_inputs(pipe, cfg, x, wl.routing(cfg), wl.router_weights(cfg))
+    pipe.mask()
+    pipe.create_indices()
+    pipe.recv_buf.fill_(0xA5)
+    pipe.dispatch_mxfp4()
+    pipe.quantize_activations()
+    torch.cuda.synchronize()
+    sep = [t.clone() for t in (pipe.recv_buf, pipe.recv_counts, pipe.xq, pipe.sfa)]
+    for t in (pipe.recv_buf, pipe.xq, pipe.sfa):
+        t.fill_(0xA5)
+    pipe.recv_counts.fill_(-1)
+    pipe.dispatch_quantize()
+    torch.cuda.synchronize()
+    for a, b, name in zip(sep, (pipe.recv_buf, pipe.recv_counts, pipe.xq, pipe.sfa),
+                          ("recv_buf", "recv_counts", "xq", "sfa")):
+        assert torch.equal(a.view(torch.uint8), b.view(torch.uint8)), name
+    # and the oracle's codes for every row
+    xq, sfa = oracle.nvfp4_quantize_bf16(x, 0.375)
+    np.testing.assert_array_equal(pipe.xq.cpu().numpy(), xq)
+    np.testing.assert_array_equal(pipe.sfa.cpu().numpy(), sfa)
+
+
 # ------------------------------------------------------------------ step 4b
 SENTINEL = 0x4B1D      # bf16 bits of an unlikely finite value (~1.03e7)
 
@@ -464,7 +498,51 @@ def test_gemv_from_the_routing_map_follows_graph_replays():
         assert_float_parity(host_bf16_f64(out)[routed], ref[routed], what="graph replay")
 
 
-def test_gemv_activation_range_is_reported():
+@pytest.mark.parametrize("path", ["grouping", "map"])
+def test_gemv_w4a16_full_bf16_range(path):
+    """W4A16 through the decode variant over bf16's whole range: tokens scaled
+    by 2^-100 .. 2^115 (about 1e-30 .. 4e34) and an outlier beyond fp16's
+    largest value in an ordinary token.  Each token's outputs, divided by its
+    power of two, meet the stated tolerance against the oracle (the absolute
+    floor alone would let tiny tokens pass trivially), and no range error is
+    raised."""
+    cfg = wl.small_config("range_full", N=32, real=32, K=1024, E=4, top_k=2, N_out=64, seed=41)
+    variant, _ = moe.moe_grouped_gemv_plan(moe.MOE_W4A16, cfg.N, cfg.top_k, cfg.E, cfg.N_out,
+                                           cfg.K)
+    assert variant == moe.MOE_GEMV_DECODE
+    xf = wl.bf16_bits_to_f32(wl.activations_bf16(cfg)).astype(np.float64)
+    exps = np.linspace(-100, 115, cfg.N).round().astype(int)
+    exps[3] = 0
+    x = xf * np.exp2(exps)[:, None]
+    x[3, 7] = 1.0e5                                   # beyond fp16 in an ordinary token
+    xb = wl.f32_to_bf16_bits(x.astype(np.float32))
+    ids = wl.routing(cfg)
+    pipe = RoutingPipeline(cfg.N, cfg.K, cfg.E, cfg.top_k, cfg.N_out, dispatch=False)
+    load_inputs(pipe, cfg, xb, ids, wl.router_weights(cfg))
+    quantize_all_weights(pipe, cfg)
+    moe.moe_get_device_error(clear=True)
+    pipe.mask()
+    pipe.create_indices()
+    pipe.expert_out.view(torch.int16).fill_(SENTINEL)
+    if path == "grouping":
+        pipe.gemv()
+    else:
+        pipe.gemv_on_map()
+    torch.cuda.synchronize()
+    assert moe.moe_get_device_error(clear=True) == 0
+    wq, sfw, gw = oracle_weights(cfg, range(cfg.E))
+    ref = oracle.grouped_gemv("w4a16", oracle.mask_padding(ids, cfg.real), wq, sfw, gw,
+                              act_bf16=xb)
+    got = host_bf16_f64(pipe.expert_out)
+    scale = np.exp2(exps.astype(np.float64))[:, None, None]
+    assert np.all(np.isfinite(got))
+    assert_float_parity(got / scale, ref / scale, what="full bf16 range (per-token scaled)")
+
+
+def test_gemv_activation_range_is_reported(monkeypatch):
+    """The tensor-memory variant feeds W4A16 activations to the tensor core as
+    fp16 without a per-token offset: a value beyond fp16's range is reported."""
+    monkeypatch.setenv("MOE_GEMV_VARIANT", "tc")
     cfg = wl.small_config("range", N=4, real=4, K=128, E=2, top_k=1, N_out=16)
     x = wl.activations_bf16(cfg)
     x[1, 5] = wl.f32_to_bf16_bits(np.array([1.0e5], np.float32))[0]   # beyond fp16 range
