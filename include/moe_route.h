@@ -76,7 +76,7 @@ typedef enum {
 /* Bits of the device error word. */
 #define MOE_DEVERR_WAIT_TIMEOUT   0x1u /* a pipeline wait in the GEMV expired           */
 #define MOE_DEVERR_RECV_OVERFLOW  0x2u /* dispatch: routed pairs exceed recv_capacity   */
-#define MOE_DEVERR_ACT_RANGE      0x4u /* W4A16 GEMV: an activation exceeds +-65504     */
+#define MOE_DEVERR_ACT_RANGE      0x4u /* W4A16 tensor-memory GEMV: |act| > 65504       */
 #define MOE_DEVERR_LIMIT          0x8u /* an internal table limit was exceeded; the call
                                           computed nothing (not expected within the
                                           documented limits)                           */
@@ -275,10 +275,13 @@ MOE_API moe_status_t moe_quantize_weights_nvfp4(const float *w, int32_t E, int32
 /* on the block-scaled FP4 tensor core (both operands stay NVFP4).  Errors: MOE_ERR_INVALID_ARG (shapes, nulls,  */
 /* alignment, a partial grouping), MOE_ERR_WORKSPACE (missing or small    */
 /* workspace when the grouping is not given); nothing is launched then.   */
-/* W4A16 activations enter the tensor cores as fp16: exact for            */
-/* 2^-14 <= |x| <= 65504, rounded to fp16 subnormals below (absolute      */
-/* error <= 2^-25); |x| > 65504 raises MOE_DEVERR_ACT_RANGE (the affected  */
-/* outputs are then undefined).                                           */
+/* W4A16 activations enter the tensor cores as fp16.  The decode variant */
+/* (moe_grouped_gemv_plan: MOE_GEMV_DECODE) scales each token by a power  */
+/* of two of its own first, so any finite bf16 token is exact down to     */
+/* 2^-29 of its largest element.  The tensor-memory variant converts      */
+/* unscaled: exact for 2^-14 <= |x| <= 65504, fp16 subnormals below       */
+/* (absolute error <= 2^-25), and |x| > 65504 raises MOE_DEVERR_ACT_RANGE */
+/* (the affected outputs are then undefined).                             */
 MOE_API size_t moe_grouped_gemv_workspace_bytes(int32_t M, int32_t top_k, int32_t E);
 MOE_API moe_status_t moe_grouped_gemv_nvfp4(moe_gemv_mode_t mode, const void *act, const uint8_t *sfa,
                                     float act_global, const int64_t *indices, int32_t M,

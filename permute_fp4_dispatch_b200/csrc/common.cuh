@@ -311,6 +311,35 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t *s
   return warp_base + x - v;
 }
 
+// As block_exclusive_scan for 64-bit values (`scratch` holds 32 of them).
+__device__ __forceinline__ uint64_t block_exclusive_scan64(uint64_t v, uint64_t *scratch,
+                                                           uint64_t *total) {
+  const unsigned lane = lane_id(), warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  uint64_t x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint64_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= (unsigned)o) x += y;
+  }
+  if (lane == 31) scratch[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    uint64_t s = lane < nw ? scratch[lane] : 0ull;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint64_t y = __shfl_up_sync(0xffffffffu, s, o);
+      if (lane >= (unsigned)o) s += y;
+    }
+    scratch[lane] = s;
+  }
+  __syncthreads();
+  const uint64_t warp_base = warp ? scratch[warp - 1] : 0ull;
+  const uint64_t t = scratch[nw - 1];
+  __syncthreads();
+  if (total) *total = t;
+  return warp_base + x - v;
+}
+
 __device__ __forceinline__ uint32_t block_max(uint32_t v, uint32_t *scratch) {
   const unsigned lane = lane_id(), warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
 #pragma unroll
@@ -449,6 +478,17 @@ __device__ __forceinline__ void cp_async16_zfill(void *dst, const void *src, uin
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_addr(dst)), "l"(src),
                "r"(src_bytes)
                : "memory");
+}
+// 1-D bulk copy (TMA engine, no multicast) of `bytes` from global to shared
+// memory, completing on an mbarrier; both addresses 16-byte aligned, bytes a
+// multiple of 16.
+__device__ __forceinline__ void bulk_load_g2s(void *dst, const void *src, uint32_t bytes,
+                                              uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_addr(dst)),
+      "l"(src), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
 }
 __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.wait_all;" ::: "memory");

@@ -34,10 +34,18 @@
 //     4 * row + line, so the swizzle key is (row & 1) * 4 + line and the eight
 //     lanes of one shared-memory phase (rows g, g + 1) hit eight distinct
 //     16-byte bank groups.
-//   * When a CTA starts a new (expert, pass), its 16 warps convert that
-//     pass's activation rows once, for the whole K, into an fp16 tile laid
-//     out in mma fragment order; every round of the pass reuses it.  W4A16:
-//     each token is scaled by a power of two of its own so that its largest
+//   * Every pair requests its first stage as soon as the CTA knows its
+//     range, so the weights stream while the CTA compacts its token lists
+//     and builds its first activation tile.
+//   * When a CTA starts a new (expert, pass), it builds that pass's fp16
+//     activation tile once, for the whole K; every round of the pass reuses
+//     it.  The tile is token-major, one row per token: W4A16 rows arrive as
+//     one bulk copy each (TMA engine, one mbarrier), then one warp per token
+//     takes the row's largest magnitude and converts the row in place, stage
+//     by stage, transposing each stage's 4 x 32 units (line t, MMA pair m) to
+//     m * 4 + t; with rows 4 units past a multiple of 8, the eight lanes of a
+//     quarter-warp read eight different bank groups.  W4A16: each
+//     token is scaled by a power of two of its own so that its largest
 //     element lands in [2^14, 2^15), then converted to fp16 -- exact for every
 //     element within 2^29 of the token's maximum, whatever the token's
 //     magnitude (bf16's whole range), and bit-identical to no scaling when the
@@ -71,13 +79,24 @@ constexpr int kStageW = kStageRows * kRowW;  // 16 KB
 constexpr int kStageSF = kStageRows * kRowSF;  // 2 KB
 constexpr int kMaxTS = 16;                   // tokens per pass at most (2 groups of 8)
 constexpr int kNG = kMaxTS / 8;
-constexpr int kGroupStageBytes = 8 * kKS * 2;  // fp16 tile of one 8-token group x one stage
-constexpr int kActBytes = 64 * 1024;
+// The fp16 activation tile is token-major: one row per token holding K
+// (rounded up to whole stages) fp16.  Within a stage the row keeps the 16-byte
+// unit of line t, MMA pair m at m * 4 + t, so that the four lanes t of one
+// token read four neighbouring units; rows are padded by 64 bytes (a row is
+// then 4 units past a multiple of 8), so the two tokens of a quarter-warp
+// fall into opposite halves of the eight 16-byte bank groups: the MMA's
+// activation loads are conflict-free.
+constexpr int kActPad = 64;
+constexpr int kActBytes = kMaxTS * (2048 * 2 + kActPad);  // 16 tokens at K = 2048
+__host__ __device__ constexpr int act_row_bytes(int K) {
+  return (K + kKS - 1) / kKS * kKS * 2 + kActPad;
+}
+static_assert((kKS * 2 / 16) % 8 == 0 && (kActPad / 16) % 8 == 4, "activation row bank layout");
 constexpr int kStagingBytes = kCW * kMaxTS * 16 * 2;
 constexpr uint64_t kActPrefetchMax = 8u << 20;     // activations prefetched into L2 up to 8 MiB
 // 16-byte activation slices per thread in a pass setup: the tile holds
-// kActBytes / 16 slices, spread over the CTA.
-constexpr int kSetupTasks = kActBytes / 16 / kThreads;
+// kActDataBytes / 16 slices, spread over the CTA.
+constexpr int kSetupTasks = kMaxTS * 2048 * 2 / 16 / kThreads;
 
 constexpr size_t kOffW = 0;
 constexpr size_t kOffSF = kOffW + (size_t)kPairs * kStageW;
@@ -100,7 +119,8 @@ constexpr size_t kOffPasses = kOffPair + kMaxTS * 4;                 // [kMaxCta
 constexpr size_t kOffPassMeta = kOffPasses + (size_t)kMaxCtaPasses * kMaxTS * 4;  // [3][kMaxCtaPasses]
 constexpr size_t kOffTokMax = kOffPassMeta + (size_t)3 * kMaxCtaPasses * 4 + 8;  // [2][kMaxTS]
 constexpr size_t kOffBar = kOffTokMax + (size_t)2 * kMaxTS * 4;
-constexpr size_t kOffMisc = kOffBar + (size_t)2 * kPairs * 8;  // full[kPairs], empty[kPairs]
+// full[kPairs], empty[kPairs], the activation rows' barrier
+constexpr size_t kOffMisc = kOffBar + (size_t)(2 * kPairs + 1) * 8;
 constexpr size_t kSmemBytes = kOffMisc + 16 + 1024;
 static_assert(kStageW % 1024 == 0, "stages must keep the 1024-byte swizzle alignment");
 static_assert(kOffBar % 8 == 0, "mbarrier alignment");
@@ -112,16 +132,10 @@ static_assert(kMaxActive <= kThreads && kStagingBytes >= (kMaxActive + 64) * 4,
 // groups (up to 2) as the activation tile holds for the whole K; 0 when not
 // even one fits.
 __host__ __device__ constexpr int tokens_per_pass(int K) {
-  const int nst = (K + kKS - 1) / kKS;
-  const int groups = kActBytes / (nst * kGroupStageBytes);
+  const int groups = kActBytes / (8 * act_row_bytes(K));
   return 8 * (groups < kNG ? groups : kNG);
 }
 
-// fp16 activation tile index (16-byte units): stage c, group G (of ng), MMA
-// pair m (MMAs 2m, 2m + 1 of the stage), lane (g, t) = 4 g + t.
-__device__ __forceinline__ int act_index(int c, int ng, int G, int m, int lane) {
-  return (((c * ng + G) * 32 + m) << 5) + lane;
-}
 
 // W4A16 tokens enter the tensor cores as fp16 scaled by a power of two of
 // their own: s = floor(log2(amax)) - 14 (clamped to [-126, 127]), so the
@@ -141,11 +155,14 @@ __device__ __forceinline__ uint32_t word_of(const uint4 &v, int i) {
 
 // One stage of one warp: lane (g, t) dequantises line t of rows g and g + 8
 // (256 codes each) and multiplies with the NG token groups of the activation
-// tile, accumulating into acc0 / acc1.
+// tile, accumulating into acc0 / acc1.  act_lane points at the stage's unit
+// (line t, pair 0) in token g's row; group G's token is 8 G rows further
+// (group_bytes apart).
 template <int NG>
-__device__ __forceinline__ void mma_stage(const uint8_t *sw, const uint8_t *ssf, const uint4 *act_c,
-                                          int g, int t, int lane, bool line_ok,
-                                          float (&acc0)[kNG][4], float (&acc1)[kNG][4]) {
+__device__ __forceinline__ void mma_stage(const uint8_t *sw, const uint8_t *ssf,
+                                          const uint8_t *act_lane, int group_bytes, int g, int t,
+                                          bool line_ok, float (&acc0)[kNG][4],
+                                          float (&acc1)[kNG][4]) {
   const uint8_t *ra = sw + g * kRowW + t * 128;
   const uint8_t *rb = ra + 8 * kRowW;
   const int key = ((g & 1) << 2) | t;  // rows g and g + 8 share the parity
@@ -179,7 +196,9 @@ __device__ __forceinline__ void mma_stage(const uint8_t *sw, const uint8_t *ssf,
       }
 #pragma unroll
       for (int G = 0; G < NG; ++G) {
-        const uint4 bv = act_c[act_index(0, NG, G, 4 * q + wd, lane)];
+        // the 8 columns of MMA pair m = 4 q + wd: codes 8 m .. 8 m + 7 of the line
+        const uint4 bv =
+            *reinterpret_cast<const uint4 *>(act_lane + G * group_bytes + (4 * q + wd) * 64);
         mma_16816_f16(acc0[G], A[0], B[0], A[1], B[1], bv.x, bv.y);
         mma_16816_f16(acc1[G], A[2], B[2], A[3], B[3], bv.z, bv.w);
       }
@@ -238,17 +257,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemv_mma_kernel(const Params p, const int ts, const __grid_constant__ CUtensorMap tmap_w,
                             const __grid_constant__ CUtensorMap tmap_sf) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint4 *act = reinterpret_cast<uint4 *>(smem + kOffAct);
+  // 1024-byte aligned by pointer arithmetic (not through an integer), so the
+  // compiler still sees shared memory and addresses it as such
+  uint8_t *smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
+  uint8_t *act = smem + kOffAct;  // token-major fp16 rows, act_row_bytes(K) apart
   uint16_t *staging = reinterpret_cast<uint16_t *>(smem + kOffStaging);
   uint32_t *prefix = reinterpret_cast<uint32_t *>(smem + kOffPrefix);
   uint32_t *s_start = reinterpret_cast<uint32_t *>(smem + kOffStart);
   int32_t *s_eid = reinterpret_cast<int32_t *>(smem + kOffEid);
   uint32_t *s_pair = reinterpret_cast<uint32_t *>(smem + kOffPair);
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + kOffBar);
+  uint64_t *act_bar = full + 2 * kPairs;  // a pass's activation rows have landed
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffMisc);
-  uint32_t *s_range = reinterpret_cast<uint32_t *>(smem + kOffMisc + 4);
 
   const int warp = threadIdx.x >> 5;
   const int lane = (int)lane_id();
@@ -259,12 +279,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&full[i], 1u);              // the leader's expect-tx arrival
       mbar_init(&full[kPairs + i], 2u);     // "empty": both warps of the pair are done
     }
+    mbar_init(act_bar, 1u);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (threadIdx.x < 2 * kMaxTS) {
     reinterpret_cast<uint32_t *>(smem + kOffTokMax)[threadIdx.x] = 0u;
   }
+  const int arow = act_row_bytes(p.K);  // bytes per token row of the tile
   if (lane == 0) {
     prefetch_tmap(&tmap_w);
     prefetch_tmap(&tmap_sf);
@@ -281,42 +303,65 @@ __global__ void __launch_bounds__(kThreads, 1)
         prefetch_l2_bulk(static_cast<const uint8_t *>(p.act) + off, min(16384u, end - off));
     }
   }
+  if (p.order == nullptr && threadIdx.x == 64 &&
+      (reinterpret_cast<uintptr_t>(p.indices) & 15u) == 0u) {
+    // the routing map this CTA will group: into L2 while the previous kernel
+    // (the mask, which may still write -1 into it) runs; a hint only (16-byte
+    // aligned maps; the size rounded down, so nothing past the map is touched)
+    const uint32_t bytes = ((uint32_t)p.M * (uint32_t)p.top_k * 8u) & ~15u;
+    for (uint32_t off = 0; off < bytes; off += 16384u)
+      prefetch_l2_bulk(reinterpret_cast<const uint8_t *>(p.indices) + off, min(16384u, bytes - off));
+  }
+  const bool fused = p.order == nullptr;
+  uint32_t *cnt = reinterpret_cast<uint32_t *>(staging);   // prologue only: expert counters
+  uint64_t *scan_scratch = reinterpret_cast<uint64_t *>(cnt + kMaxActive);  // and scan scratch
+  if (fused) {  // the counters are this CTA's own: cleared while the previous grid runs
+    for (int e = threadIdx.x; e < p.E; e += kThreads) cnt[e] = 0u;
+    __syncthreads();
+  }
   pdl_wait();
   pdl_launch_dependents();
   const int N = p.N, K = p.K;
   const int RB = (N + 15) / 16;
-  const bool fused = p.order == nullptr;
-  uint32_t *cnt = reinterpret_cast<uint32_t *>(staging);   // prologue only: expert counters
-  uint32_t *scan_scratch = cnt + kMaxActive;               // and block-scan scratch
   int32_t my_ids[kFusedPer];  // in-kernel grouping: experts of this thread's slots (-1: none)
   const int fq = fused ? (p.M * p.top_k + kThreads - 1) / kThreads : 0;
-  uint32_t A;
+  uint32_t A, U;
   if (fused) {
     // group the routing map here: counts per expert, then the active experts in
     // ascending id with their CSR offsets (the moe_create_indices definition)
+    // and the row-block units before each (its passes times RB)
     const int S = p.M * p.top_k;
-    for (int e = threadIdx.x; e < p.E; e += kThreads) cnt[e] = 0u;
 #pragma unroll
     for (int j = 0; j < kFusedPer; ++j) {
       const int slot = (int)threadIdx.x * fq + j;
       const int64_t id = (j < fq && slot < S) ? __ldg(p.indices + slot) : -1;
       my_ids[j] = (id >= 0 && id < p.E) ? (int32_t)id : -1;
     }
-    __syncthreads();
 #pragma unroll
     for (int j = 0; j < kFusedPer; ++j)
       if (my_ids[j] >= 0) atomicAdd(&cnt[my_ids[j]], 1u);
     __syncthreads();
+    // one scan of (passes << 32 | active flag << 16 | count): counts stay below
+    // 2^13 and the active experts below 2^10, so no field carries into the next
     const uint32_t c = (int)threadIdx.x < p.E ? cnt[threadIdx.x] : 0u;
-    uint32_t n_active, n_routed;
-    const uint32_t pos = block_exclusive_scan(c > 0u ? 1u : 0u, scan_scratch, &n_active);
-    const uint32_t off = block_exclusive_scan(c, scan_scratch, &n_routed);
+    const uint32_t passes = (c + (uint32_t)ts - 1u) / (uint32_t)ts;
+    uint64_t tot;
+    const uint64_t sc = block_exclusive_scan64(
+        ((uint64_t)passes << 32) | (c > 0u ? 0x10000u : 0u) | c, scan_scratch, &tot);
+    const uint32_t pos = ((uint32_t)sc >> 16) & 0xFFFFu, off = (uint32_t)sc & 0xFFFFu;
+    const uint32_t n_active = ((uint32_t)tot >> 16) & 0xFFFFu, n_routed = (uint32_t)tot & 0xFFFFu;
     if (c > 0u) {
       s_eid[pos] = (int32_t)threadIdx.x;
       s_start[pos] = off;
+      prefix[pos] = (uint32_t)(sc >> 32) * (uint32_t)RB;
     }
-    if (threadIdx.x == 0) s_start[n_active] = n_routed;
+    if (threadIdx.x == 0) {
+      s_start[n_active] = n_routed;
+      prefix[n_active] = (uint32_t)(tot >> 32) * (uint32_t)RB;
+    }
     A = n_active;
+    U = (uint32_t)(tot >> 32) * (uint32_t)RB;
+    __syncthreads();
   } else {
     A = p.stats[1];
     // the grouping of the active experts (at most kMaxActive, checked on the host)
@@ -325,25 +370,68 @@ __global__ void __launch_bounds__(kThreads, 1)
       s_start[i] = p.start[i];
       if (i < A) s_eid[i] = p.eids[i];
     }
+    __syncthreads();
+    if (warp == 0) build_prefix(prefix, s_start, A, (uint32_t)ts, RB, lane);
+    __syncthreads();
+    U = prefix[A];
   }
-  __syncthreads();
-  if (warp == 0) {
-    build_prefix(prefix, s_start, A, (uint32_t)ts, RB, lane);
-    __syncwarp();
-    if (lane == 0) {  // the CTA's share of the units, computed once
-      uint32_t u0, u1;
-      cta_pass_range(prefix[A], RB, kCW, u0, u1);
-      s_range[0] = u0;
-      s_range[1] = u1;
-    }
-  }
-  __syncthreads();
-
-  const uint32_t u_begin = s_range[0], u_end = s_range[1];
+  // the CTA's share of the units (every thread computes the same)
+  uint32_t u_begin, u_end;
+  cta_pass_range(U, RB, kCW, u_begin, u_end);
   if (u_begin >= u_end) return;
   const int nst = (K + kKS - 1) / kKS;  // stages per block
   const int lines_total = K / 256;
   const Meta meta{prefix, s_start, s_eid, N};
+  int pass_idx = -1;  // index of the current pass in s_passes
+  uint32_t act_issued = 0;  // passes whose row copies warp 0 has requested (lane 0's count)
+  const int pair = warp >> 1, half = warp & 1;
+  const bool leader = half == 0;  // the pair's even warp issues the pair's copies
+  uint8_t *pw = smem + kOffW + (size_t)pair * kStageW;
+  uint8_t *ps = smem + kOffSF + (size_t)pair * kStageSF;
+  uint64_t *pfull = full + pair;
+  uint64_t *pempty = full + kPairs + pair;
+
+  // ---- producer side of the pair's pipeline (leader warp): the next (round, stage)
+  // in which the pair holds a block
+  RoundWalk piter;
+  piter.init(meta, A, RB, u_begin, u_end);
+  Round pr;
+  int pc = 0;
+  bool pvalid = false;
+  auto next_own_round = [&]() {
+    pvalid = false;
+    pc = 0;
+    while (piter.next(meta, RB, (uint32_t)ts, pr))
+      if (2 * pair < pr.nblk) {
+        pvalid = true;
+        break;
+      }
+  };
+  next_own_round();
+  uint32_t produced = 0;
+  auto produce = [&]() {
+    // lane 0's view of the abort flag decides for the whole warp
+    if (!leader || !pvalid || __shfl_sync(0xFFFFFFFFu, *abort_flag, 0)) return;
+    // the stage is refilled once both warps of the pair have released its previous contents
+    if (produced > 0 && !mbar_wait_bounded(pempty, (produced - 1) & 1u, p.wait_limit_ns))
+      *abort_flag = 1;
+    if (__shfl_sync(0xFFFFFFFFu, *abort_flag, 0)) return;
+    const int n0 = pr.n0 + 32 * pair;
+    if (lane == 0) {
+      const uint64_t policy = l2_evict_first_policy();  // made here: no register holds it between stages
+      mbar_arrive_expect_tx(pfull, (uint32_t)(kStageW + kStageSF));
+      tma_load_4d(pw, &tmap_w, 0, pc * kLines, n0, pr.e, pfull, policy);
+      // scales: 32 rows x 4 words (one 16-byte group per line), rows beyond N and
+      // lines beyond K read as zero
+      tma_load_3d(ps, &tmap_sf, pc * kLines * 4, n0, pr.e, pfull, policy);
+    }
+    ++produced;
+    if (++pc == nst) next_own_round();
+  };
+  // the first stage of every pair is requested as soon as the range is known:
+  // the weights stream while the CTA gathers its token lists and activations
+  produce();
+
   uint32_t *s_passes = reinterpret_cast<uint32_t *>(smem + kOffPasses);
   int n_passes = 0;
   if (fused) {
@@ -381,7 +469,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t mine = 0, total;
 #pragma unroll
       for (int j = 0; j < kFusedPer; ++j) mine += my_ids[j] == e ? 1u : 0u;
-      uint32_t rank = block_exclusive_scan(mine, scan_scratch, &total);
+      uint32_t rank = block_exclusive_scan(mine, reinterpret_cast<uint32_t *>(scan_scratch), &total);
 #pragma unroll
       for (int j = 0; j < kFusedPer; ++j) {
         if (my_ids[j] != e) continue;
@@ -393,54 +481,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncthreads();
   }
-  int pass_idx = -1;  // index of the current pass in s_passes
-  const int pair = warp >> 1, half = warp & 1;
-  const bool leader = half == 0;  // the pair's even warp issues the pair's copies
-  uint8_t *pw = smem + kOffW + (size_t)pair * kStageW;
-  uint8_t *ps = smem + kOffSF + (size_t)pair * kStageSF;
-  uint64_t *pfull = full + pair;
-  uint64_t *pempty = full + kPairs + pair;
-  const uint64_t policy = l2_evict_first_policy();
-
-  // ---- producer side of the pair's pipeline (leader warp): the next (round, stage)
-  // in which the pair holds a block
-  RoundWalk piter;
-  piter.init(meta, A, RB, u_begin, u_end);
-  Round pr;
-  int pc = 0;
-  bool pvalid = false;
-  auto next_own_round = [&]() {
-    pvalid = false;
-    pc = 0;
-    while (piter.next(meta, RB, (uint32_t)ts, pr))
-      if (2 * pair < pr.nblk) {
-        pvalid = true;
-        break;
-      }
-  };
-  next_own_round();
-  uint32_t produced = 0;
-  auto produce = [&]() {
-    // lane 0's view of the abort flag decides for the whole warp
-    if (!leader || !pvalid || __shfl_sync(0xFFFFFFFFu, *abort_flag, 0)) return;
-    // the stage is refilled once both warps of the pair have released its previous contents
-    if (produced > 0 && !mbar_wait_bounded(pempty, (produced - 1) & 1u, p.wait_limit_ns))
-      *abort_flag = 1;
-    if (__shfl_sync(0xFFFFFFFFu, *abort_flag, 0)) return;
-    const int n0 = pr.n0 + 32 * pair;
-    if (lane == 0) {
-      mbar_arrive_expect_tx(pfull, (uint32_t)(kStageW + kStageSF));
-      tma_load_4d(pw, &tmap_w, 0, pc * kLines, n0, pr.e, pfull, policy);
-      // scales: 32 rows x 4 words (one 16-byte group per line), rows beyond N and
-      // lines beyond K read as zero
-      tma_load_3d(ps, &tmap_sf, pc * kLines * 4, n0, pr.e, pfull, policy);
-    }
-    ++produced;
-    if (++pc == nst) next_own_round();
-  };
-  // the first stages are requested right after the first pass's activation
-  // loads, so the small gathers are not queued behind the weight stream
-  bool primed = false;
 
   // ---- consumer side
   const int g = lane >> 2, t = lane & 3;
@@ -454,17 +494,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   while (iter.next(meta, RB, (uint32_t)ts, r)) {
     if (r.tok0 != pass_key) {
-      // ---- new (expert, pass): build its fp16 activation tile for the whole K.
-      // The loads (token order, then activation slices) are issued before the
-      // barrier that frees the previous tile, so their latency overlaps it.
-      // Task b of a thread is slice kk of token tau, task = b * kThreads + tid =
-      // tau * per_tok + kk.  per_tok is a multiple of 32, so tau is the same
-      // across a warp, and lane j of every warp holds the row of token j.
-      const int per_tok = kpad / 8;  // 8-column slices per token
-      const int ntask = r.ntok * per_tok;  // at most kSetupTasks * kThreads
-      const int tau0 = (int)threadIdx.x / per_tok, kk0 = (int)threadIdx.x - tau0 * per_tok;
-      uint4 v[kSetupTasks];
-      uint32_t sv[kSetupTasks];
+      // ---- new (expert, pass): build its fp16 activation tile for the whole K,
+      // one row per token (lane j of every warp holds the pair of token j)
       uint32_t my_pair = 0, my_row = 0;
       ++pass_idx;
       // (the host's limits keep a CTA's passes within the table; should one
@@ -478,86 +509,113 @@ __global__ void __launch_bounds__(kThreads, 1)
         my_pair = fused ? s_passes[pass_idx * kMaxTS + lane] : __ldg(p.order + r.tok0 + lane);
         my_row = my_pair / (uint32_t)p.top_k;
       }
-      int tau = tau0, kk = kk0;
-#pragma unroll
-      for (int b = 0; b < kSetupTasks; ++b) {
-        const int task = b * kThreads + (int)threadIdx.x;
-        const int64_t m = (int64_t)__shfl_sync(0xFFFFFFFFu, my_row, tau & 31);
-        const int k = kk * 8;
-        v[b] = make_uint4(0u, 0u, 0u, 0u);
-        sv[b] = 0u;
-        if (task < ntask) {
-          if (k < K) {
-            if (MODE == MOE_W4A16) {
-              v[b] = ldg_nc_v4(static_cast<const uint16_t *>(p.act) + m * K + k);
-            } else {
-              const uint8_t *qp = static_cast<const uint8_t *>(p.act) + m * (K / 2);
-              v[b].x = __ldg(reinterpret_cast<const uint32_t *>(qp + k / 2));
-              sv[b] = p.sfa[m * (K / 16) + k / 16];
-            }
-          }
-        }
-        for (kk += kThreads; kk >= per_tok; kk -= per_tok) ++tau;
-      }
-      // W4A16: every token's largest magnitude (a warp's lanes share a token per
-      // task, so one atomic per warp and task), into this pass's buffer
       uint32_t *tokmax = reinterpret_cast<uint32_t *>(smem + kOffTokMax) + (pass_idx & 1) * kMaxTS;
+      const int ng_new = (r.ntok + 7) / 8;
       if (MODE == MOE_W4A16) {
-        int tm = tau0;
-        int km = kk0;
-#pragma unroll
-        for (int b = 0; b < kSetupTasks; ++b) {
-          const int task = b * kThreads + (int)threadIdx.x;
-          const int tk = tm;
-          for (km += kThreads; km >= per_tok; km -= per_tok) ++tm;
-          if (task - (int)lane >= ntask) continue;  // warp-uniform: the whole warp is past the tasks
+        // the previous tile is free once every warp is here
+        if (pass_key != 0xFFFFFFFFu) named_bar_sync(1, kThreads);
+        // each token's bf16 row, one bulk copy straight into its tile row
+        if (warp == 0 && !__shfl_sync(0xFFFFFFFFu, *abort_flag, 0)) {
+          // the previous pass's plain reads and writes of the tile come before
+          // the copies' writes
+          fence_proxy_async_smem();
+          if (lane == 0) {
+            mbar_arrive_expect_tx(act_bar, (uint32_t)r.ntok * (uint32_t)K * 2u);
+            ++act_issued;
+          }
+          __syncwarp();
+          if (lane < r.ntok)
+            bulk_load_g2s(act + lane * arow, static_cast<const uint16_t *>(p.act) + (int64_t)my_row * K,
+                          (uint32_t)K * 2u, act_bar);
+        }
+        if (!*abort_flag && !mbar_wait_bounded(act_bar, (uint32_t)pass_idx & 1u, p.wait_limit_ns))
+          *abort_flag = 1;
+        if (warp < r.ntok) {
+          // one warp per token row: the row's largest magnitude, then each
+          // stage converted in place -- scaled by the token's power of two
+          // (exact), fp16 (exact in range) -- and its 4 x 32 units (line t,
+          // pair m) transposed to m * 4 + t; columns past K become zeros
+          uint8_t *row = act + warp * arow;
+          const int units = K / 8;
           uint32_t mx = 0u;
-          if (task < ntask) {
-            const uint32_t w4[4] = {v[b].x, v[b].y, v[b].z, v[b].w};
+          for (int u = lane; u < units; u += 32) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(row + u * 16);
+            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
             for (int i = 0; i < 4; ++i)
               mx = max(mx, max((w4[i] << 16) & 0x7FFF0000u, w4[i] & 0x7FFF0000u));
           }
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-          if (lane == 0 && mx) atomicMax(&tokmax[tk], mx);
+          if (lane == 0) tokmax[warp] = mx;
+          const float down = pow2f(-token_shift(mx));
+          for (int c = 0; c < nst; ++c) {
+            uint4 h[4];
+#pragma unroll
+            for (int tl = 0; tl < 4; ++tl) {
+              const int u = c * (kKS / 8) + tl * 32 + lane;
+              h[tl] = make_uint4(0u, 0u, 0u, 0u);
+              if (u < units) {
+                const uint4 v = *reinterpret_cast<const uint4 *>(row + u * 16);
+                float f[8];
+                f[0] = bf16_lo(v.x); f[1] = bf16_hi(v.x);
+                f[2] = bf16_lo(v.y); f[3] = bf16_hi(v.y);
+                f[4] = bf16_lo(v.z); f[5] = bf16_hi(v.z);
+                f[6] = bf16_lo(v.w); f[7] = bf16_hi(v.w);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) f[e] = __fmul_rn(f[e], down);
+                h[tl] = make_uint4(pack_f16x2(f[0], f[1]), pack_f16x2(f[2], f[3]),
+                                   pack_f16x2(f[4], f[5]), pack_f16x2(f[6], f[7]));
+              }
+            }
+            __syncwarp();  // the stage's units are all read before any is rewritten
+#pragma unroll
+            for (int tl = 0; tl < 4; ++tl)
+              *reinterpret_cast<uint4 *>(row + (c * (kKS / 8) + lane * 4 + tl) * 16) = h[tl];
+            __syncwarp();
+          }
         }
-      }
-      if (!primed) {
-        produce();
-        primed = true;
-      }
-      if (pass_key != 0xFFFFFFFFu) named_bar_sync(1, kThreads);  // previous tile no longer read
-      // the other maxima buffer served the previous pass, which is done: clear it for the next
-      if (MODE == MOE_W4A16 && (int)threadIdx.x < kMaxTS)
-        reinterpret_cast<uint32_t *>(smem + kOffTokMax)[((pass_idx + 1) & 1) * kMaxTS + threadIdx.x] = 0u;
-      ng = (r.ntok + 7) / 8;
-      if ((int)threadIdx.x < r.ntok) s_pair[threadIdx.x] = my_pair;
-      tau = tau0;
-      kk = kk0;
+        ng = ng_new;
+        if ((int)threadIdx.x < r.ntok) s_pair[threadIdx.x] = my_pair;
+      } else {
+        // W4A4: the NVFP4 codes and their scales are loaded before the barrier
+        // that frees the previous tile, so their latency overlaps it; columns
+        // past K (up to the last stage's end) are written as zeros.  Task b of
+        // a thread is slice kk of token tau, b * kThreads + tid = tau * per_tok
+        // + kk; per_tok is a multiple of 32, so tau is the same across a warp.
+        const int per_tok = kpad / 8;  // 8-column slices per token
+        const int ntask = r.ntok * per_tok;  // at most kSetupTasks * kThreads
+        const int tau0 = (int)threadIdx.x / per_tok, kk0 = (int)threadIdx.x - tau0 * per_tok;
+        int tau = tau0, kk = kk0;
+        uint4 v[kSetupTasks];
+        uint32_t sv[kSetupTasks];
 #pragma unroll
-      for (int b = 0; b < kSetupTasks; ++b) {
-        const int task = b * kThreads + (int)threadIdx.x;
-        const int tk = tau, k = kk * 8;
-        for (kk += kThreads; kk >= per_tok; kk -= per_tok) ++tau;
-        if (task >= ntask) continue;
-        uint4 hv = make_uint4(0u, 0u, 0u, 0u);
-        if (k < K) {
-          if (MODE == MOE_W4A16) {
-            // scaled by the token's power of two (exact), then fp16 (exact in range)
-            const float down = pow2f(-token_shift(tokmax[tk]));
-            float f[8];
-            f[0] = bf16_lo(v[b].x); f[1] = bf16_hi(v[b].x);
-            f[2] = bf16_lo(v[b].y); f[3] = bf16_hi(v[b].y);
-            f[4] = bf16_lo(v[b].z); f[5] = bf16_hi(v[b].z);
-            f[6] = bf16_lo(v[b].w); f[7] = bf16_hi(v[b].w);
+        for (int b = 0; b < kSetupTasks; ++b) {
+          const int task = b * kThreads + (int)threadIdx.x;
+          const int64_t m = (int64_t)__shfl_sync(0xFFFFFFFFu, my_row, tau & 31);
+          const int k = kk * 8;
+          v[b] = make_uint4(0u, 0u, 0u, 0u);
+          sv[b] = 0u;
+          if (task < ntask && k < K) {
+            const uint8_t *qp = static_cast<const uint8_t *>(p.act) + m * (K / 2);
+            v[b].x = __ldg(reinterpret_cast<const uint32_t *>(qp + k / 2));
+            sv[b] = p.sfa[m * (K / 16) + k / 16];
+          }
+          for (kk += kThreads; kk >= per_tok; kk -= per_tok) ++tau;
+        }
+        if (pass_key != 0xFFFFFFFFu) named_bar_sync(1, kThreads);  // previous tile no longer read
+        ng = ng_new;
+        if ((int)threadIdx.x < r.ntok) s_pair[threadIdx.x] = my_pair;
+        tau = tau0;
+        kk = kk0;
 #pragma unroll
-            for (int e = 0; e < 8; ++e) f[e] = __fmul_rn(f[e], down);
-            hv.x = pack_f16x2(f[0], f[1]);
-            hv.y = pack_f16x2(f[2], f[3]);
-            hv.z = pack_f16x2(f[4], f[5]);
-            hv.w = pack_f16x2(f[6], f[7]);
-          } else {
+        for (int b = 0; b < kSetupTasks; ++b) {
+          const int task = b * kThreads + (int)threadIdx.x;
+          const int tk = tau, k = kk * 8;
+          for (kk += kThreads; kk >= per_tok; kk -= per_tok) ++tau;
+          if (task >= ntask) continue;
+          uint4 hv = make_uint4(0u, 0u, 0u, 0u);
+          if (k < K) {
             const uint32_t sc = bcast_lo(e4m3x2_to_f16x2(sv[b]));
             uint32_t q0, q1, q2, q3;
             e2m1x8_to_f16x2(v[b].x, q0, q1, q2, q3);
@@ -566,10 +624,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             hv.z = hmul2(q2, sc);
             hv.w = hmul2(q3, sc);
           }
+          // columns [k, k + 8): stage c, line lt, MMA pair m, kept at unit m * 4 + lt
+          const int u = k / 8, c = u / (kKS / 8), lt = (u % (kKS / 8)) / 32, m = u % 32;
+          *reinterpret_cast<uint4 *>(act + tk * arow + (c * (kKS / 8) + m * 4 + lt) * 16) = hv;
         }
-        // columns [k, k + 8): stage c, line lt, MMA pair m of lane (tk % 8, lt)
-        const int c = k / kKS, kc = k % kKS, lt = kc / 256, m = (kc % 256) / 8;
-        act[act_index(c, ng, tk / 8, m, (tk & 7) * 4 + lt)] = hv;
       }
       named_bar_sync(1, kThreads);
       pass_key = r.tok0;
@@ -592,11 +650,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint8_t *sw = pw + (size_t)half * 16 * kRowW;
         const uint8_t *ssf = ps + (size_t)half * 16 * kRowSF;
         const bool line_ok = c * kLines + t < lines_total;
-        const uint4 *act_c = act + act_index(c, ng, 0, 0, 0);
+        const uint8_t *act_lane = act + g * arow + c * (kKS * 2) + t * 16;
         if (ng == 1)
-          mma_stage<1>(sw, ssf, act_c, g, t, lane, line_ok, acc0, acc1);
+          mma_stage<1>(sw, ssf, act_lane, 8 * arow, g, t, line_ok, acc0, acc1);
         else
-          mma_stage<2>(sw, ssf, act_c, g, t, lane, line_ok, acc0, acc1);
+          mma_stage<2>(sw, ssf, act_lane, 8 * arow, g, t, line_ok, acc0, acc1);
       }
       ++consumed;
       __syncwarp();  // every lane is done with the stage
@@ -647,10 +705,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
-  // After a timed-out wait, let the pair's copies still in flight land
-  // before the CTA exits (bounded again).
+  // After a timed-out wait, let the copies still in flight land before the
+  // CTA exits (bounded again).
   if (*abort_flag && leader && lane == 0 && produced > 0)
     mbar_wait_bounded(pfull, (produced - 1) & 1u, kDrainLimitNs);
+  if (*abort_flag && warp == 0 && lane == 0 && act_issued > 0)
+    mbar_wait_bounded(act_bar, (act_issued - 1) & 1u, kDrainLimitNs);
 }
 
 }  // namespace mma

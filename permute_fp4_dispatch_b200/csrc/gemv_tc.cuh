@@ -86,8 +86,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   pdl_wait();
   pdl_launch_dependents();
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  // 1024-byte aligned by pointer arithmetic (not through an integer), so the
+  // compiler still sees shared memory and addresses it as such
+  uint8_t *smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
   uint8_t *btile = smem + kOffB;
   uint32_t *prefix = reinterpret_cast<uint32_t *>(smem + kOffPrefix);
   uint32_t *s_start = reinterpret_cast<uint32_t *>(smem + kOffStart);
