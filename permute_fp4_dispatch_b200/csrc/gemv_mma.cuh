@@ -443,7 +443,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t *pf = reinterpret_cast<uint32_t *>(pe + kMaxCtaPasses);
     int32_t *pn = reinterpret_cast<int32_t *>(pf + kMaxCtaPasses);
     int32_t *s_np = pn + kMaxCtaPasses;
-    if (threadIdx.x == 0) {
+    if (U / (uint32_t)RB <= gridDim.x) {
+      // no more passes than CTAs: the range lies in one pass, which every
+      // thread finds by itself (the shared copy serves the pass set-up)
+      const int a = expert_of_unit(prefix, A, u_begin);
+      const uint32_t pass = (u_begin - prefix[a]) / (uint32_t)RB;
+      const uint32_t c = s_start[a + 1] - s_start[a];
+      const int32_t e = s_eid[a];
+      const uint32_t first = pass * (uint32_t)ts;
+      const int ntok = (int)min((uint32_t)ts, c - first);
+      uint32_t mine = 0, total;
+#pragma unroll
+      for (int j = 0; j < kFusedPer; ++j) mine += my_ids[j] == e ? 1u : 0u;
+      uint32_t rank = block_exclusive_scan(mine, reinterpret_cast<uint32_t *>(scan_scratch), &total);
+#pragma unroll
+      for (int j = 0; j < kFusedPer; ++j) {
+        if (my_ids[j] != e) continue;
+        if (rank - first < (uint32_t)ntok)
+          s_passes[rank - first] = (uint32_t)threadIdx.x * (uint32_t)fq + (uint32_t)j;
+        ++rank;
+      }
+      n_passes = 1;
+    } else if (threadIdx.x == 0) {
       RoundWalk w;
       w.init(meta, A, RB, u_begin, u_end);
       Round rr;
@@ -460,23 +481,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       *s_np = cnt_p;
     }
-    __syncthreads();
-    const int np = *s_np;
-    n_passes = np;
-    for (int i = 0; i < np; ++i) {
-      if (i > 0 && pe[i] == pe[i - 1]) continue;  // the passes of one expert share a scan
-      const int e = pe[i];
-      uint32_t mine = 0, total;
+    if (n_passes == 0) {
+      __syncthreads();
+      const int np = *s_np;
+      n_passes = np;
+      for (int i = 0; i < np; ++i) {
+        if (i > 0 && pe[i] == pe[i - 1]) continue;  // the passes of one expert share a scan
+        const int e = pe[i];
+        uint32_t mine = 0, total;
 #pragma unroll
-      for (int j = 0; j < kFusedPer; ++j) mine += my_ids[j] == e ? 1u : 0u;
-      uint32_t rank = block_exclusive_scan(mine, reinterpret_cast<uint32_t *>(scan_scratch), &total);
+        for (int j = 0; j < kFusedPer; ++j) mine += my_ids[j] == e ? 1u : 0u;
+        uint32_t rank =
+            block_exclusive_scan(mine, reinterpret_cast<uint32_t *>(scan_scratch), &total);
 #pragma unroll
-      for (int j = 0; j < kFusedPer; ++j) {
-        if (my_ids[j] != e) continue;
-        for (int k = i; k < np && pe[k] == e; ++k)
-          if (rank - pf[k] < (uint32_t)pn[k])
-            s_passes[k * kMaxTS + (rank - pf[k])] = (uint32_t)threadIdx.x * (uint32_t)fq + (uint32_t)j;
-        ++rank;
+        for (int j = 0; j < kFusedPer; ++j) {
+          if (my_ids[j] != e) continue;
+          for (int k = i; k < np && pe[k] == e; ++k)
+            if (rank - pf[k] < (uint32_t)pn[k])
+              s_passes[k * kMaxTS + (rank - pf[k])] =
+                  (uint32_t)threadIdx.x * (uint32_t)fq + (uint32_t)j;
+          ++rank;
+        }
       }
     }
     __syncthreads();
