@@ -76,7 +76,7 @@ typedef enum {
 /* Bits of the device error word. */
 #define MOE_DEVERR_WAIT_TIMEOUT   0x1u /* a pipeline wait in the GEMV expired           */
 #define MOE_DEVERR_RECV_OVERFLOW  0x2u /* dispatch: routed pairs exceed recv_capacity   */
-#define MOE_DEVERR_ACT_RANGE      0x4u /* W4A16 tensor-memory GEMV: |act| > 65504       */
+#define MOE_DEVERR_ACT_RANGE      0x4u /* W4A16 GEMV without offsets: |act| > 65504     */
 #define MOE_DEVERR_LIMIT          0x8u /* an internal table limit was exceeded; the call
                                           computed nothing (not expected within the
                                           documented limits)                           */
@@ -265,24 +265,31 @@ MOE_API moe_status_t moe_quantize_weights_nvfp4(const float *w, int32_t E, int32
 /*             expert_usage_stats: EITHER all four, the moe_create_indices */
 /*             outputs for this same map (then indices may be NULL), OR   */
 /*             all four NULL: the call then groups the pairs of indices   */
-/*             itself (one extra launch) into `workspace`, which must hold */
-/*             moe_grouped_gemv_workspace_bytes(M, top_k, E) bytes, 256-  */
-/*             byte aligned, caller-owned, contents need no initialisation */
-/*             (with the grouping given, workspace may be NULL)           */
+/*             itself (one extra launch) into `workspace`                 */
+/*   workspace caller-owned device memory, 256-byte aligned, contents need */
+/*             no initialisation; moe_grouped_gemv_workspace_bytes(M,     */
+/*             top_k, E, K) bytes serve every variant.  Its first part    */
+/*             holds the grouping (required when the grouping is not      */
+/*             given); the rest holds the W4A16 activations converted     */
+/*             once per call for the tensor-memory variant (used when it  */
+/*             fits; with the grouping given that part starts at offset   */
+/*             0 and workspace may be NULL)                               */
 /* "M = routed pairs, top_k = 1" is simply a routing map of shape [R, 1]. */
 /* Limits: K % 32 == 0, N % 8 == 0, 1 <= top_k <= E <= 1024; act, w, sfw  */
-/* and out 16-byte aligned, sfa 4-byte aligned.  W4A4 with K % 64 == 0 runs */
-/* on the block-scaled FP4 tensor core (both operands stay NVFP4).  Errors: MOE_ERR_INVALID_ARG (shapes, nulls,  */
-/* alignment, a partial grouping), MOE_ERR_WORKSPACE (missing or small    */
-/* workspace when the grouping is not given); nothing is launched then.   */
-/* W4A16 activations enter the tensor cores as fp16.  The decode variant */
-/* (moe_grouped_gemv_plan: MOE_GEMV_DECODE) scales each token by a power  */
-/* of two of its own first, so any finite bf16 token is exact down to     */
-/* 2^-29 of its largest element.  The tensor-memory variant converts      */
-/* unscaled: exact for 2^-14 <= |x| <= 65504, fp16 subnormals below       */
-/* (absolute error <= 2^-25), and |x| > 65504 raises MOE_DEVERR_ACT_RANGE */
-/* (the affected outputs are then undefined).                             */
-MOE_API size_t moe_grouped_gemv_workspace_bytes(int32_t M, int32_t top_k, int32_t E);
+/* and out 16-byte aligned, sfa 4-byte aligned.  W4A4 with K % 64 == 0    */
+/* runs on the block-scaled FP4 tensor core (both operands stay NVFP4).   */
+/* Errors: MOE_ERR_INVALID_ARG (shapes, nulls, alignment, a partial       */
+/* grouping), MOE_ERR_WORKSPACE (missing or small workspace when the      */
+/* grouping is not given); nothing is launched then.                      */
+/* W4A16 activations enter the tensor cores as fp16, each token that does */
+/* not already fit fp16 exactly scaled by a power of two of its own first */
+/* (the epilogue multiplies it back), so any finite bf16 token is exact   */
+/* down to 2^-29 of its largest element.  Only a tensor-memory call whose */
+/* workspace lacks the room for the converted activations converts them   */
+/* chunk by chunk without offsets: exact for 2^-14 <= |x| <= 65504, fp16  */
+/* subnormals below (absolute error <= 2^-25), and |x| > 65504 raises     */
+/* MOE_DEVERR_ACT_RANGE (the affected outputs are then undefined).        */
+MOE_API size_t moe_grouped_gemv_workspace_bytes(int32_t M, int32_t top_k, int32_t E, int32_t K);
 MOE_API moe_status_t moe_grouped_gemv_nvfp4(moe_gemv_mode_t mode, const void *act, const uint8_t *sfa,
                                     float act_global, const int64_t *indices, int32_t M,
                                     int32_t top_k, const uint8_t *w, const uint8_t *sfw,

@@ -68,7 +68,7 @@ _SIGS = {
     "moe_dispatch_mxfp4_quantize_nvfp4": ([_P, _I32, _I32, _I32, _I32, _P, _P, _P, _P, _P, _I64,
                                            _P, _F32, _P, _P, _P], _I32),
     "moe_quantize_weights_nvfp4": ([_P, _I32, _I32, _I32, _P, _P, _P, _P], _I32),
-    "moe_grouped_gemv_workspace_bytes": ([_I32, _I32, _I32], _SZ),
+    "moe_grouped_gemv_workspace_bytes": ([_I32, _I32, _I32, _I32], _SZ),
     "moe_grouped_gemv_nvfp4": ([_I32, _P, _P, _F32, _P, _I32, _I32, _P, _P, _P, _I32, _I32, _I32,
                                 _P, _P, _P, _P, _P, _P, _SZ, _P], _I32),
     "moe_grouped_gemv_plan": ([_I32, _I32, _I32, _I32, _I32, _I32, _I32, _P, _P], _I32),
@@ -212,8 +212,8 @@ def moe_quantize_weights_nvfp4(w, E: int, N: int, K: int, wq, sfw, w_global, str
         "moe_quantize_weights_nvfp4")
 
 
-def moe_grouped_gemv_workspace_bytes(M: int, top_k: int, E: int) -> int:
-    return library().moe_grouped_gemv_workspace_bytes(M, top_k, E)
+def moe_grouped_gemv_workspace_bytes(M: int, top_k: int, E: int, K: int) -> int:
+    return library().moe_grouped_gemv_workspace_bytes(M, top_k, E, K)
 
 
 def moe_grouped_gemv_nvfp4(mode: int, act, sfa, act_global: float, indices, M: int, top_k: int,
@@ -221,8 +221,10 @@ def moe_grouped_gemv_nvfp4(mode: int, act, sfa, act_global: float, indices, M: i
                            expert_start_indices=None, expert_ids=None, expert_usage_stats=None,
                            out=None, workspace=None, ws_bytes: int = 0, stream=None):
     """Grouped GEMV over the routing map ``indices`` [M, top_k].  Pass the
-    four moe_create_indices outputs for this map, or none of them and a
-    workspace of moe_grouped_gemv_workspace_bytes(M, top_k, E) bytes."""
+    four moe_create_indices outputs for this map, or none of them; a workspace
+    of moe_grouped_gemv_workspace_bytes(M, top_k, E, K) bytes serves every
+    variant (required without the grouping; with it, W4A16 in the
+    tensor-memory variant converts its activations there once)."""
     _check(library().moe_grouped_gemv_nvfp4(
         mode, _ptr(act), _ptr(sfa), act_global, _ptr(indices), M, top_k, _ptr(w), _ptr(sfw),
         _ptr(w_global), E, N, K, _ptr(token_expert_order), _ptr(expert_start_indices),

@@ -137,17 +137,6 @@ __host__ __device__ constexpr int tokens_per_pass(int K) {
 }
 
 
-// W4A16 tokens enter the tensor cores as fp16 scaled by a power of two of
-// their own: s = floor(log2(amax)) - 14 (clamped to [-126, 127]), so the
-// token's largest element lands in [2^14, 2^15) and every bf16 value of the
-// token within 2^29 of it is exact in fp16.  amax_bits are the fp32 bits of
-// the token's largest magnitude.
-__device__ __forceinline__ int token_shift(uint32_t amax_bits) {
-  if (amax_bits == 0u) return 0;
-  int s = (int)((amax_bits >> 23) & 0xFFu) - 127 - 14;
-  return s < -126 ? -126 : (s > 127 ? 127 : s);
-}
-__device__ __forceinline__ float pow2f(int s) { return __uint_as_float((uint32_t)(s + 127) << 23); }
 
 __device__ __forceinline__ uint32_t word_of(const uint4 &v, int i) {
   return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;

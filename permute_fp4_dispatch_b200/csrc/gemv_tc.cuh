@@ -38,10 +38,15 @@
 //     D is double-buffered in TMEM, so a round's epilogue (tcgen05.ld, scale
 //     by g_w * g_a, round to bf16, store) runs while the next round's first
 //     chunk is already being multiplied.
-//   * W4A16 activations enter the tensor core as fp16: exact for
-//     2^-14 <= |x| <= 65504, fp16-subnormal rounding (absolute error
-//     <= 2^-25) below; |x| > 65504 raises MOE_DEVERR_ACT_RANGE.  W4A4
-//     activations are dequantised exactly like the weights.
+//   * W4A16 activations enter the tensor core as fp16.  Given room in the
+//     caller's workspace, act_f16_kernel converts them once per call, each
+//     token that does not fit fp16 exactly scaled by a power of two of its
+//     own (exact over bf16's whole range, the power multiplied back in the
+//     epilogue), and the staging warps only copy them.  Otherwise each chunk
+//     is converted as it is staged: exact for 2^-14 <= |x| <= 65504,
+//     fp16-subnormal rounding (absolute error <= 2^-25) below; |x| > 65504
+//     raises MOE_DEVERR_ACT_RANGE.  W4A4 activations are dequantised
+//     exactly like the weights.
 #pragma once
 #include "gemv_common.cuh"
 
@@ -74,15 +79,68 @@ constexpr size_t kOffPrefix = kOffB + 2 * kBTile;
 constexpr size_t kOffStart = kOffPrefix + (kMaxExperts + 4) * 4;
 constexpr size_t kOffEid = kOffStart + (kMaxExperts + 4) * 4;
 constexpr size_t kOffPair = kOffEid + (kMaxExperts + 4) * 4;     // [2][kTS] pair ids
-constexpr size_t kOffBar = kOffPair + 2 * kTS * 4;
+constexpr size_t kOffShift = kOffPair + 2 * kTS * 4;  // [2][kTS] W4A16 token offsets
+constexpr size_t kOffBar = kOffShift + 2 * kTS * 4;
 constexpr int kNumBars = 2 * kStages + 9;
 constexpr size_t kOffMisc = kOffBar + kNumBars * 8;             // tmem slot, abort flag
 constexpr size_t kSmemBytes = kOffMisc + 16 + 1024;             // + alignment slack
 
+// W4A16 activations converted once per call for this variant (it stages
+// activations for every 128-row round and 256-column chunk, so converting
+// them there would repeat the work per round): one warp per row m of act,
+// shift[m] = 0 when the row already converts to fp16 exactly (every nonzero
+// magnitude within [2^-14, 65504]), else token_shift(its largest magnitude);
+// act16 row m = fp16(act row m * 2^-shift[m]) (exact: a power of two).
+__global__ void __launch_bounds__(256)
+    act_f16_kernel(const uint16_t *__restrict__ act, int32_t M, int32_t K,
+                   int32_t *__restrict__ shift, uint16_t *__restrict__ act16) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int m = (int)blockIdx.x * 8 + (int)(threadIdx.x >> 5);
+  const unsigned lane = lane_id();
+  if (m >= M) return;
+  const uint16_t *row = act + (int64_t)m * K;
+  uint32_t mx = 0u, mn = 0xFFFFFFFFu;  // fp32 bits of the largest and smallest nonzero magnitude
+  for (int k = 8 * (int)lane; k < K; k += 256) {  // K % 32 == 0: whole 16-byte slices
+    const uint4 v = ldg_nc_v4(row + k);
+    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t lo = (w4[i] << 16) & 0x7FFF0000u, hi = w4[i] & 0x7FFF0000u;
+      mx = max(mx, max(lo, hi));
+      mn = min(mn, min(lo ? lo : 0xFFFFFFFFu, hi ? hi : 0xFFFFFFFFu));
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+  }
+  // 0x477FE000 = 65504 (fp16's largest), 0x38800000 = 2^-14 (its smallest normal)
+  const bool fits = mx <= 0x477FE000u && (mn == 0xFFFFFFFFu || mn >= 0x38800000u);
+  const int sh = fits ? 0 : token_shift(mx);
+  if (lane == 0) shift[m] = sh;
+  const float down = pow2f(-sh);
+  uint16_t *out = act16 + (int64_t)m * K;
+  for (int k = 8 * (int)lane; k < K; k += 256) {
+    const uint4 v = ldg_nc_v4(row + k);
+    float f[8];
+    f[0] = bf16_lo(v.x); f[1] = bf16_hi(v.x);
+    f[2] = bf16_lo(v.y); f[3] = bf16_hi(v.y);
+    f[4] = bf16_lo(v.z); f[5] = bf16_hi(v.z);
+    f[6] = bf16_lo(v.w); f[7] = bf16_hi(v.w);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) f[e] = __fmul_rn(f[e], down);
+    *reinterpret_cast<uint4 *>(out + k) = make_uint4(pack_f16x2(f[0], f[1]), pack_f16x2(f[2], f[3]),
+                                                     pack_f16x2(f[4], f[5]), pack_f16x2(f[6], f[7]));
+  }
+}
+
 template <int MODE, bool SF_TMA>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemv_kernel(const Params p, const __grid_constant__ CUtensorMap tmap_w,
-                        const __grid_constant__ CUtensorMap tmap_sf) {
+                        const __grid_constant__ CUtensorMap tmap_sf,
+                        const uint16_t *__restrict__ act16, const int32_t *__restrict__ act_shift) {
   pdl_wait();
   pdl_launch_dependents();
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -94,6 +152,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t *s_start = reinterpret_cast<uint32_t *>(smem + kOffStart);
   int32_t *s_eid = reinterpret_cast<int32_t *>(smem + kOffEid);
   uint32_t *s_pair = reinterpret_cast<uint32_t *>(smem + kOffPair);
+  int32_t *s_shift = reinterpret_cast<int32_t *>(smem + kOffShift);
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + kOffBar);
   uint64_t *empty = full + kStages;
   uint64_t *a_full = empty + kStages;   // [2]
@@ -262,11 +321,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     // token pair ids of the current / next round, one token per lane (lanes < 8):
     // lane i of warp w holds token tau = w + 8 i
     uint32_t pair_cur = 0xFFFFFFFFu, pair_nxt = 0xFFFFFFFFu;
-    auto fetch_pairs = [&](const Round &q_, uint32_t &dst) {
+    int32_t sh_cur = 0, sh_nxt = 0;  // the same tokens' W4A16 offsets (0 without act16)
+    const bool pre = MODE == MOE_W4A16 && act16 != nullptr;  // activations converted already
+    auto fetch_pairs = [&](const Round &q_, uint32_t &dst, int32_t &sh) {
       const int tau = warp + 8 * lane;
       dst = (lane < 8 && tau < q_.ntok) ? p.order[q_.tok0 + tau] : 0xFFFFFFFFu;
+      sh = (pre && dst != 0xFFFFFFFFu) ? act_shift[dst / (uint32_t)p.top_k] : 0;
     };
-    if (have) fetch_pairs(r, pair_cur);
+    if (have) fetch_pairs(r, pair_cur, sh_cur);
 
     // activations of this warp's tokens for one chunk (8 values per lane per token)
     uint4 raw[8];
@@ -281,7 +343,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (warp + 8 * i < ntok && kv) {
           const int64_t m = (int64_t)(pr / (uint32_t)p.top_k);
           if (MODE == MOE_W4A16) {
-            raw[i] = ldg_nc_v4(static_cast<const uint16_t *>(p.act) + m * K + k0 + 8 * lane);
+            raw[i] = ldg_nc_v4((pre ? act16 : static_cast<const uint16_t *>(p.act)) + m * K + k0 +
+                               8 * lane);
           } else {
             const uint8_t *qp = static_cast<const uint8_t *>(p.act) + m * (K / 2);
             raw[i].x = __ldg(reinterpret_cast<const uint32_t *>(qp + (k0 + 8 * lane) / 2));
@@ -319,12 +382,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float f = __fmul_rn(gw, p.g_a);
         const int n = er.n0 + row;
         const uint32_t *pairs = s_pair + (ernd & 1u) * kTS;
+        const int32_t *shifts = s_shift + (ernd & 1u) * kTS;
         const int ncol = min(32, er.ntok - c0);
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           if (i < ncol) {
             const uint32_t pr = pairs[c0 + i];
-            const __nv_bfloat16 o = __float2bfloat16_rn(__uint_as_float(v[i]) * f);
+            float y = __fmul_rn(__uint_as_float(v[i]), f);
+            // the token's power of two last (no early overflow, the same
+            // rounding as without the offset)
+            const int sh = shifts[c0 + i];
+            if (sh != 0) y = __fmul_rn(y, pow2f(sh));  // warp-uniform: one column per i
+            const __nv_bfloat16 o = __float2bfloat16_rn(y);
             p.out[(int64_t)pr * N + n] = __bfloat16_as_ushort(o);
           }
         }
@@ -334,9 +403,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     while (have) {
       // ---- round start: publish this round's pair ids, fetch the next round's
       named_bar_sync(1, kDQ * 32);
-      if (lane < 8 && warp + 8 * lane < r.ntok)
+      if (lane < 8 && warp + 8 * lane < r.ntok) {
         s_pair[(rnd & 1u) * kTS + warp + 8 * lane] = pair_cur;
-      if (have_n) fetch_pairs(rn, pair_nxt);
+        s_shift[(rnd & 1u) * kTS + warp + 8 * lane] = sh_cur;
+      }
+      if (have_n) fetch_pairs(rn, pair_nxt, sh_nxt);
       named_bar_sync(1, kDQ * 32);
       const bool has_rows = 32 * q < r.nrows;
 
@@ -392,7 +463,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int tau = warp + 8 * i;
           if (tau >= r.ntok) continue;  // warp-uniform
           uint4 hv;
-          if (MODE == MOE_W4A16) {
+          if (pre) {
+            hv = raw[i];  // fp16 already, scaled by the token's power of two
+          } else if (MODE == MOE_W4A16) {
             float f[8];
             f[0] = bf16_lo(raw[i].x); f[1] = bf16_hi(raw[i].x);
             f[2] = bf16_lo(raw[i].y); f[3] = bf16_hi(raw[i].y);
@@ -444,6 +517,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++rnd;
       r = rn;
       pair_cur = pair_nxt;
+      sh_cur = sh_nxt;
       have = have_n;
       have_n = have && iter.next(meta, RB, rn);
     }

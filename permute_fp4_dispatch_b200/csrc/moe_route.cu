@@ -535,6 +535,23 @@ GemvGrouping gemv_grouping_layout(int64_t S, int32_t E, void *base) {
   g.total = off;
   return g;
 }
+
+// The W4A16 activations converted once per call (tensor-memory variant):
+// per-token offsets [M] int32, then the fp16 rows [M, K].
+struct GemvActF16 {
+  int32_t *shift;
+  uint16_t *act16;
+  size_t total;
+};
+GemvActF16 gemv_act_f16_layout(int64_t M, int64_t K, void *base) {
+  GemvActF16 a{};
+  uint8_t *b = static_cast<uint8_t *>(base);
+  a.shift = b ? reinterpret_cast<int32_t *>(b) : nullptr;
+  const size_t off = round256((size_t)M * 4);
+  a.act16 = b ? reinterpret_cast<uint16_t *>(b + off) : nullptr;
+  a.total = off + round256((size_t)M * (size_t)K * 2);
+  return a;
+}
 }  // namespace
 
 namespace {
@@ -574,9 +591,10 @@ GemvPlan plan_gemv(moe_gemv_mode_t mode, int64_t S, int32_t E, int32_t K, bool g
 }
 }  // namespace
 
-size_t moe_grouped_gemv_workspace_bytes(int32_t M, int32_t top_k, int32_t E) {
-  if (M < 0 || top_k < 1 || E < 1) return 0;
-  return gemv_grouping_layout((int64_t)M * top_k, E, nullptr).total;
+size_t moe_grouped_gemv_workspace_bytes(int32_t M, int32_t top_k, int32_t E, int32_t K) {
+  if (M < 0 || top_k < 1 || E < 1 || K < 0) return 0;
+  return gemv_grouping_layout((int64_t)M * top_k, E, nullptr).total +
+         gemv_act_f16_layout(M, K, nullptr).total;
 }
 
 moe_status_t moe_grouped_gemv_nvfp4(moe_gemv_mode_t mode, const void *act, const uint8_t *sfa,
@@ -618,6 +636,17 @@ moe_status_t moe_grouped_gemv_nvfp4(moe_gemv_mode_t mode, const void *act, const
   if (M == 0) return MOE_OK;
   const GemvPlan plan = plan_gemv(mode, S, E, K, given == 4, sms);
   const bool fused_grouping = plan.groups_in_kernel;
+  // W4A16 in the tensor-memory variant converts the activations once, into
+  // the workspace after the grouping's sections (at its start when the
+  // grouping is given), when the workspace has room for them
+  GemvActF16 a16{};
+  if (mode == MOE_W4A16 && plan.variant == MOE_GEMV_TENSOR_MEMORY && workspace &&
+      aligned(workspace, 256)) {
+    const size_t base = given == 0 ? gemv_grouping_layout(S, E, nullptr).total : 0;
+    const GemvActF16 need = gemv_act_f16_layout(M, K, nullptr);
+    if (ws_bytes >= base + need.total)
+      a16 = gemv_act_f16_layout(M, K, static_cast<uint8_t *>(workspace) + base);
+  }
   if (given == 0 && !fused_grouping) {
     // group the pairs of the routing map first, into the caller's workspace
     const GemvGrouping g = gemv_grouping_layout(S, E, workspace);
@@ -670,7 +699,13 @@ moe_status_t moe_grouped_gemv_nvfp4(moe_gemv_mode_t mode, const void *act, const
     return launch_pdl(kern, dim3((unsigned)sms), dim3(mma::kThreads), mma::kSmemBytes, s, p,
                       ts_mma, maps.tlines, maps.tsf_lines);
   }
-  void (*kern)(const Params, const CUtensorMap, const CUtensorMap);
+  if (a16.act16) {
+    st = launch_pdl(tc::act_f16_kernel, dim3((unsigned)((M + 7) / 8)), dim3(256), 0, s,
+                    static_cast<const uint16_t *>(act), M, K, a16.shift, a16.act16);
+    if (st != MOE_OK) return st;
+  }
+  void (*kern)(const Params, const CUtensorMap, const CUtensorMap, const uint16_t *,
+               const int32_t *);
   if (mode == MOE_W4A16)
     kern = maps.sf_tma ? tc::grouped_gemv_kernel<MOE_W4A16, true>
                        : tc::grouped_gemv_kernel<MOE_W4A16, false>;
@@ -679,7 +714,8 @@ moe_status_t moe_grouped_gemv_nvfp4(moe_gemv_mode_t mode, const void *act, const
                        : tc::grouped_gemv_kernel<MOE_W4A4, false>;
   if ((st = set_smem(kern, tc::kSmemBytes)) != MOE_OK) return st;
   return launch_pdl(kern, dim3((unsigned)sms), dim3(tc::kThreads), tc::kSmemBytes, s, p, maps.tw,
-                    maps.tsf);
+                    maps.tsf, static_cast<const uint16_t *>(a16.act16),
+                    static_cast<const int32_t *>(a16.shift));
 }
 
 moe_status_t moe_grouped_gemv_plan(moe_gemv_mode_t mode, int32_t M, int32_t top_k, int32_t E,

@@ -15,7 +15,8 @@ from __future__ import annotations
 
 import torch
 
-from . import (MOE_EPI_IDENTITY, MOE_EPI_NONE, MOE_EPI_SCALE, MOE_W4A4, MOE_W4A16,
+from . import (MOE_EPI_IDENTITY, MOE_EPI_NONE, MOE_EPI_SCALE, MOE_GEMV_TENSOR_MEMORY,
+               MOE_W4A4, MOE_W4A16,
                moe_combine, moe_create_indices, moe_create_indices_workspace_bytes,
                moe_mask_and_create_indices, moe_grouped_gemv_plan,
                moe_grouped_gemv_workspace_bytes,
@@ -104,8 +105,9 @@ class RoutingPipeline:
         else:
             self.xq = self.sfa = None
         self.expert_out = torch.zeros((N, top_k, N_out), dtype=torch.bfloat16, device=dev)
-        # the GEMV's own grouping workspace (used when it is handed the map alone)
-        self.gemv_ws_bytes = moe_grouped_gemv_workspace_bytes(N, top_k, E)
+        # the GEMV's workspace: its grouping (when handed the map alone) and, for W4A16
+        # in the tensor-memory variant, the activations converted once
+        self.gemv_ws_bytes = moe_grouped_gemv_workspace_bytes(N, top_k, E, K)
         self.gemv_ws = torch.empty(max(self.gemv_ws_bytes, 256), dtype=u8, device=dev)
         # Step order of run():
         #   "gemv_groups"   mask -> GEMV on the routing map (the GEMV groups the
@@ -117,6 +119,9 @@ class RoutingPipeline:
         # map itself (decode-sized W4A16), so grouping is off its critical path.
         _, in_kernel = moe_grouped_gemv_plan(self.gemv_mode, N, top_k, E, N_out, K)
         self.order = "gemv_groups" if in_kernel else "routing_first"
+        # the variant the routing_first order's GEMV (grouping given) runs
+        self.gemv_variant, _ = moe_grouped_gemv_plan(self.gemv_mode, N, top_k, E, N_out, K,
+                                                     grouping_given=True)
         # W4A4 in the "routing_first" order: the MXFP4 dispatch and the NVFP4
         # activation quantisation as one kernel (one read of x) before the GEMV
         self.fuse_dispatch_quant = self.gemv_mode == MOE_W4A4 and dispatch
@@ -191,7 +196,8 @@ class RoutingPipeline:
                                self.N, self.top_k, self.wq, self.sfw, self.w_global, self.E,
                                self.N_out, self.K, self.token_expert_order,
                                self.expert_start_indices, self.expert_ids,
-                               self.expert_usage_stats, self.expert_out, stream=stream)
+                               self.expert_usage_stats, self.expert_out, workspace=self.gemv_ws,
+                               ws_bytes=self.gemv_ws_bytes, stream=stream)
 
     def gemv_on_map(self, stream=None):
         """The GEMV on the routing map alone (it groups the pairs itself)."""
@@ -338,6 +344,8 @@ class RoutingPipeline:
             n = 1 + ci + 1                       # mask, create_indices, GEMV (groups in-kernel)
         else:
             n = (1 if self.S <= 1024 else 1 + ci) + 1
+            if self.gemv_mode == MOE_W4A16 and self.gemv_variant == MOE_GEMV_TENSOR_MEMORY:
+                n += 1                           # the activations' fp16 conversion
         if self.order == "routing_first" and self.fuse_dispatch_quant:
             n += 1
         else:

@@ -66,7 +66,8 @@ def test_host_validation_runs_before_any_device_work(lib):
                 None) == 1                                                            # partial grouping
     assert gemv(0, P, None, 1.0, None, 4, 2, P, P, None, 4, 16, 64, None, None, None, None, P,
                 None, 0, None) == 1                                                   # no map at all
-    ws = moe.moe_grouped_gemv_workspace_bytes(4, 2, 4)
+    # the grouping's part of the workspace (the rest holds converted activations)
+    ws = moe.moe_grouped_gemv_workspace_bytes(4, 2, 4, 64) - 256 - 512
     assert gemv(0, P, None, 1.0, P, 4, 2, P, P, None, 4, 16, 64, None, None, None, None, P,
                 P * 16, ws - 1, None) == 3                                            # workspace size
     assert gemv(0, P, None, 1.0, P, 4, 2, P, P, None, 4, 16, 64, None, None, None, None, P,
@@ -82,11 +83,13 @@ def test_workspace_sizing(lib):
     assert moe.moe_mxfp4_row_stride(2048) == 1088
     assert moe.moe_mxfp4_row_stride(2880) == 1536
     # grouped GEMV workspace: order, restore [S] u32, starts [E+1], ids [E], stats [2],
-    # then the grouping call's own workspace, each section 256-byte aligned
+    # the grouping call's own workspace, then W4A16 activations converted once
+    # (per-token offsets [M] int32, fp16 rows [M, K]), each section 256-byte aligned
     r = lambda n: -(-n // 256) * 256  # noqa: E731
-    S, E = 1024, 128
-    assert moe.moe_grouped_gemv_workspace_bytes(128, 8, 128) == (
-        2 * r(4 * S) + r(4 * (E + 1)) + r(4 * E) + r(8) + 256)
-    S, E = 98304, 64
-    assert moe.moe_grouped_gemv_workspace_bytes(16384, 6, 64) == (
-        2 * r(4 * S) + r(4 * (E + 1)) + r(4 * E) + r(8) + r(256 + 12 * 64 * 4))
+    S, E, M, K = 1024, 128, 128, 2048
+    assert moe.moe_grouped_gemv_workspace_bytes(M, 8, E, K) == (
+        2 * r(4 * S) + r(4 * (E + 1)) + r(4 * E) + r(8) + 256 + r(4 * M) + r(2 * M * K))
+    S, E, M, K = 98304, 64, 16384, 4096
+    assert moe.moe_grouped_gemv_workspace_bytes(M, 6, E, K) == (
+        2 * r(4 * S) + r(4 * (E + 1)) + r(4 * E) + r(8) + r(256 + 12 * 64 * 4) + r(4 * M) +
+        r(2 * M * K))

@@ -411,7 +411,7 @@ def test_gemv_from_the_routing_map_alone(mode, gemv_variant):
     the same bits as the call that is handed the grouping."""
     cfg = wl.small_config("bare", N=50, real=44, K=512, E=7, top_k=4, N_out=136)
     pipe, x, ids = run_gemv_case(cfg, mode)
-    ws = torch.full((moe.moe_grouped_gemv_workspace_bytes(cfg.N, cfg.top_k, cfg.E),), 0x5A,
+    ws = torch.full((moe.moe_grouped_gemv_workspace_bytes(cfg.N, cfg.top_k, cfg.E, cfg.K),), 0x5A,
                     dtype=torch.uint8, device="cuda")
     out = torch.empty_like(pipe.expert_out)
     out.view(torch.int16).fill_(SENTINEL)
@@ -472,7 +472,7 @@ def test_gemv_from_the_routing_map_follows_graph_replays():
     written between replays."""
     cfg = wl.small_config("bare_graph", N=40, real=40, K=256, E=6, top_k=2, N_out=64)
     pipe, x, _ = run_gemv_case(cfg, "w4a16")
-    ws = torch.empty(moe.moe_grouped_gemv_workspace_bytes(cfg.N, cfg.top_k, cfg.E),
+    ws = torch.empty(moe.moe_grouped_gemv_workspace_bytes(cfg.N, cfg.top_k, cfg.E, cfg.K),
                      dtype=torch.uint8, device="cuda")
     out = torch.empty_like(pipe.expert_out)
     s = torch.cuda.Stream()
@@ -498,18 +498,22 @@ def test_gemv_from_the_routing_map_follows_graph_replays():
         assert_float_parity(host_bf16_f64(out)[routed], ref[routed], what="graph replay")
 
 
+@pytest.mark.parametrize("variant", ["auto", "tc"])
 @pytest.mark.parametrize("path", ["grouping", "map"])
-def test_gemv_w4a16_full_bf16_range(path):
-    """W4A16 through the decode variant over bf16's whole range: tokens scaled
-    by 2^-100 .. 2^115 (about 1e-30 .. 4e34) and an outlier beyond fp16's
-    largest value in an ordinary token.  Each token's outputs, divided by its
-    power of two, meet the stated tolerance against the oracle (the absolute
-    floor alone would let tiny tokens pass trivially), and no range error is
-    raised."""
+def test_gemv_w4a16_full_bf16_range(path, variant, monkeypatch):
+    """W4A16 over bf16's whole range, in the decode variant (the plan's
+    choice here) and the tensor-memory variant (its activations converted
+    once into the workspace): tokens scaled by 2^-100 .. 2^115 (about 1e-30
+    .. 4e34) and an outlier beyond fp16's largest value in an ordinary token.
+    Each token's outputs, divided by its power of two, meet the stated
+    tolerance against the oracle (the absolute floor alone would let tiny
+    tokens pass trivially), and no range error is raised."""
+    if variant != "auto":
+        monkeypatch.setenv("MOE_GEMV_VARIANT", variant)
     cfg = wl.small_config("range_full", N=32, real=32, K=1024, E=4, top_k=2, N_out=64, seed=41)
-    variant, _ = moe.moe_grouped_gemv_plan(moe.MOE_W4A16, cfg.N, cfg.top_k, cfg.E, cfg.N_out,
-                                           cfg.K)
-    assert variant == moe.MOE_GEMV_DECODE
+    got, _ = moe.moe_grouped_gemv_plan(moe.MOE_W4A16, cfg.N, cfg.top_k, cfg.E, cfg.N_out, cfg.K,
+                                       grouping_given=(path == "grouping"))
+    assert got == (moe.MOE_GEMV_DECODE if variant == "auto" else moe.MOE_GEMV_TENSOR_MEMORY)
     xf = wl.bf16_bits_to_f32(wl.activations_bf16(cfg)).astype(np.float64)
     exps = np.linspace(-100, 115, cfg.N).round().astype(int)
     exps[3] = 0
@@ -540,8 +544,9 @@ def test_gemv_w4a16_full_bf16_range(path):
 
 
 def test_gemv_activation_range_is_reported(monkeypatch):
-    """The tensor-memory variant feeds W4A16 activations to the tensor core as
-    fp16 without a per-token offset: a value beyond fp16's range is reported."""
+    """Called with the grouping and no workspace, the tensor-memory variant
+    converts W4A16 activations chunk by chunk without per-token offsets: a
+    value beyond fp16's range is reported."""
     monkeypatch.setenv("MOE_GEMV_VARIANT", "tc")
     cfg = wl.small_config("range", N=4, real=4, K=128, E=2, top_k=1, N_out=16)
     x = wl.activations_bf16(cfg)
@@ -552,7 +557,10 @@ def test_gemv_activation_range_is_reported(monkeypatch):
     assert moe.moe_get_device_error(clear=True) == 0
     pipe.mask()
     pipe.create_indices()
-    pipe.gemv()
+    moe.moe_grouped_gemv_nvfp4(moe.MOE_W4A16, pipe.x, None, 1.0, pipe.routing_map, cfg.N,
+                               cfg.top_k, pipe.wq, pipe.sfw, pipe.w_global, cfg.E, cfg.N_out, cfg.K,
+                               pipe.token_expert_order, pipe.expert_start_indices,
+                               pipe.expert_ids, pipe.expert_usage_stats, pipe.expert_out)
     assert moe.moe_get_device_error(clear=True) & moe.MOE_DEVERR_ACT_RANGE
 
 
