@@ -11,11 +11,14 @@
 //
 // Design (one persistent CTA per SM, 6 warps):
 //   * Work units are (active expert a, 128-row block rb, pass p of up to
-//     kTS = 128 tokens), in that order, so the passes of one row block follow
+//     kTS tokens), in that order, so the passes of one row block follow
 //     each other and a block's weights are read from HBM once even when its
 //     expert holds more tokens than one pass.  The CTAs take equal contiguous
 //     ranges of units.  One unit is one MMA tile: M = 128 weight rows (A),
 //     N = the pass's tokens rounded up to 16 (B), fp32 D in tensor memory.
+//     kTS = 128 with 5 stages in flight, or -- when the experts hold 64
+//     tokens or fewer on average -- kTS = 64, whose smaller token tiles leave
+//     room for 7 stages (more weight bytes in flight per SM).
 //   * warp 0, lane 0: streams the unit's weight codes, 128 rows x 256 codes
 //     per stage, with one TMA box (128B swizzle, L2 evict-first; rows past N
 //     and codes past K arrive as zeros) into a kStages-deep ring;
@@ -50,28 +53,34 @@ constexpr int kSWThreads = 4 * 32;
 constexpr int kThreads = 2 * 32 + kSWThreads;
 constexpr int kKC = 256;                  // codes per stage: 128 bytes of each row
 constexpr int kKSteps = kKC / 64;         // MMAs (K = 64) per stage
-constexpr int kTS = 128;                  // tokens per pass
-constexpr int kStages = 5;
 constexpr int kATile = 128 * 128;         // weight tile: 128 rows x 128 bytes
-constexpr int kBTile = kTS * 128;         // token tile: 128 rows x 128 bytes
 constexpr int kSFStep = 512;              // one operand's scales for one MMA: 32 rows x 16 B
 constexpr int kSFBytes = kKSteps * kSFStep;
-constexpr int kStageBytes = kATile + kBTile + 2 * kSFBytes;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kDcol = 0;             // D: two buffers of kTS columns
-constexpr uint32_t kSFcol = 2 * kTS;      // per stage: 16 columns of A scales, 16 of B scales
-static_assert(kSFcol + kStages * 32 <= kTmemCols, "tensor memory columns");
-static_assert(kStageBytes % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
 
-constexpr size_t kOffStart = (size_t)kStages * kStageBytes;
-constexpr size_t kOffEid = kOffStart + (kMaxExperts + 4) * 4;
-constexpr size_t kOffPrefix = kOffEid + (kMaxExperts + 4) * 4;
-constexpr size_t kOffPair = kOffPrefix + (kMaxExperts + 4) * 4;  // [2][kTS] pair ids
-constexpr size_t kOffBar = kOffPair + 2 * kTS * 4;
-constexpr int kNumBars = 3 * kStages + 5;
-constexpr size_t kOffMisc = kOffBar + kNumBars * 8;              // tmem slot, abort flag
-constexpr size_t kSmemBytes = kOffMisc + 16 + 1024;              // + alignment slack
-static_assert(kSmemBytes <= 232448, "shared memory per block");
+// Sizes for TS tokens per pass: 128 (many tokens per expert), or 64 -- a
+// smaller token tile leaves room for two more stages, i.e. more weight
+// bytes in flight per SM, which experts with few tokens need.
+template <int TS>
+struct Cfg {
+  static constexpr int kTS = TS;                        // tokens per pass (MMA N <= TS)
+  static constexpr int kStages = TS >= 128 ? 5 : 7;
+  static constexpr int kBTile = TS * 128;               // token tile: TS rows x 128 bytes
+  static constexpr int kStageBytes = kATile + kBTile + 2 * kSFBytes;
+  static constexpr uint32_t kSFcol = 2 * TS;            // per stage: 16 columns of A scales, 16 of B
+  static constexpr size_t kOffStart = (size_t)kStages * kStageBytes;
+  static constexpr size_t kOffEid = kOffStart + (kMaxExperts + 4) * 4;
+  static constexpr size_t kOffPrefix = kOffEid + (kMaxExperts + 4) * 4;
+  static constexpr size_t kOffPair = kOffPrefix + (kMaxExperts + 4) * 4;  // [2][kTS] pair ids
+  static constexpr size_t kOffBar = kOffPair + 2 * TS * 4;
+  static constexpr int kNumBars = 3 * kStages + 5;
+  static constexpr size_t kOffMisc = kOffBar + kNumBars * 8;             // tmem slot, abort flag
+  static constexpr size_t kSmemBytes = kOffMisc + 16 + 1024;             // + alignment slack
+  static_assert(kSFcol + kStages * 32 <= kTmemCols, "tensor memory columns");
+  static_assert(kStageBytes % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
+  static_assert(kSmemBytes <= 232448, "shared memory per block");
+};
 
 struct Unit {
   int e;          // expert id
@@ -82,6 +91,7 @@ struct Unit {
 
 // Walks a CTA's unit range in order; unit u of active expert a with c pairs
 // (P = ceil(c / kTS) passes) is block v / P, pass v % P, v = u - prefix[a].
+template <int kTS>
 struct UnitWalk {
   uint32_t u, u_end;
   int a;
@@ -102,8 +112,15 @@ struct UnitWalk {
   }
 };
 
+template <int TS>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemv_bs_kernel(const Params p, const __grid_constant__ CUtensorMap tmap_w) {
+  using C = Cfg<TS>;
+  constexpr int kTS = C::kTS, kStages = C::kStages, kBTile = C::kBTile;
+  constexpr int kStageBytes = C::kStageBytes;
+  constexpr uint32_t kSFcol = C::kSFcol;
+  constexpr size_t kOffStart = C::kOffStart, kOffEid = C::kOffEid, kOffPrefix = C::kOffPrefix;
+  constexpr size_t kOffPair = C::kOffPair, kOffBar = C::kOffBar, kOffMisc = C::kOffMisc;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -171,7 +188,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ================================================================ weight tiles (TMA)
     if (lane == 0) {
       const uint64_t policy = l2_evict_first_policy();
-      UnitWalk walk{u0, u1, a0};
+      UnitWalk<kTS> walk{u0, u1, a0};
       Unit r;
       uint32_t it = 0, issued = 0;
       while (!*abort_flag && walk.next(prefix, s_start, s_eid, r)) {
@@ -196,7 +213,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kMmaWarp) {
     // ================================================================ MMA issuer
     if (lane == 0) {
-      UnitWalk walk{u0, u1, a0};
+      UnitWalk<kTS> walk{u0, u1, a0};
       Unit r;
       uint32_t it = 0, rnd = 0;
       while (walk.next(prefix, s_start, s_eid, r)) {
@@ -243,7 +260,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q = warp & 3;                       // the TMEM lane quadrant this warp may access
     const int64_t xrow = K / 2, sfrow = K / 16;
     const uint8_t *xq = static_cast<const uint8_t *>(p.act);
-    UnitWalk walk{u0, u1, a0};
+    UnitWalk<kTS> walk{u0, u1, a0};
     Unit r, rp;
     bool have = walk.next(prefix, s_start, s_eid, r), pending = false;
     uint32_t it = 0, rnd = 0, rnd_p = 0;

@@ -94,8 +94,9 @@ __host__ __device__ constexpr int act_row_bytes(int K) {
 static_assert((kKS * 2 / 16) % 8 == 0 && (kActPad / 16) % 8 == 4, "activation row bank layout");
 constexpr int kStagingBytes = kCW * kMaxTS * 16 * 2;
 constexpr uint64_t kActPrefetchMax = 8u << 20;     // activations prefetched into L2 up to 8 MiB
-// 16-byte activation slices per thread in a pass setup: the tile holds
-// kActDataBytes / 16 slices, spread over the CTA.
+// 16-byte activation slices per thread in a W4A4 pass set-up: a tile holds
+// ts rows of act_row_bytes(K) <= kActBytes, so ts * kpad <= 16 * 2048
+// columns, 8 columns per slice, spread over the CTA.
 constexpr int kSetupTasks = kMaxTS * 2048 * 2 / 16 / kThreads;
 
 constexpr size_t kOffW = 0;

@@ -687,9 +687,14 @@ moe_status_t moe_grouped_gemv_nvfp4(moe_gemv_mode_t mode, const void *act, const
   const bool use_mma = plan.variant == MOE_GEMV_DECODE;
   const int ts_mma = use_mma ? mma::tokens_per_pass(K) : 0;
   if (use_bs) {
-    if ((st = set_smem(bs::grouped_gemv_bs_kernel, bs::kSmemBytes)) != MOE_OK) return st;
-    return launch_pdl(bs::grouped_gemv_bs_kernel, dim3((unsigned)sms), dim3(bs::kThreads),
-                      bs::kSmemBytes, s, p, maps.tbs);
+    // passes of 64 tokens (two more stages in flight) when the experts hold
+    // 64 tokens or fewer on average, else 128
+    const bool small = S <= (int64_t)64 * E;
+    void (*kern)(const Params, const CUtensorMap) =
+        small ? bs::grouped_gemv_bs_kernel<64> : bs::grouped_gemv_bs_kernel<128>;
+    const size_t smem = small ? bs::Cfg<64>::kSmemBytes : bs::Cfg<128>::kSmemBytes;
+    if ((st = set_smem(kern, smem)) != MOE_OK) return st;
+    return launch_pdl(kern, dim3((unsigned)sms), dim3(bs::kThreads), smem, s, p, maps.tbs);
   }
   if (use_mma) {
     void (*kern)(const Params, const int, const CUtensorMap, const CUtensorMap) =
