@@ -21,11 +21,15 @@
 //     room for 7 stages (more weight bytes in flight per SM).
 //   * warp 0, lane 0: streams the unit's weight codes, 128 rows x 256 codes
 //     per stage, with one TMA box (128B swizzle, L2 evict-first; rows past N
-//     and codes past K arrive as zeros) into a kStages-deep ring;
+//     and codes past K arrive as zeros) into a kStages-deep ring, and -- when
+//     the scale rows are whole 16-byte units (K % 256 == 0) -- the stage's
+//     weight scales as a second box, row-major;
 //   * warps 2-5 (128 threads): per stage, gather the pass's token rows
 //     (128 bytes of codes each) into the 128B-swizzled K-major B tile, and
 //     the stage's scale factors of both operands into shared memory in the
-//     tensor core's 32-row x 16-byte scale layout, all with cp.async laid
+//     tensor core's 32-row x 16-byte scale layout (the weight scales, when
+//     they came by TMA, moved there from the row-major box: one 16-byte
+//     load and four 4-byte stores per row), all with cp.async laid
 //     out so one warp instruction covers whole rows (no copies for rows the
 //     result does not use), arriving on the stage's barrier when the copies
 //     land; they also run the epilogue
@@ -56,18 +60,22 @@ constexpr int kKSteps = kKC / 64;         // MMAs (K = 64) per stage
 constexpr int kATile = 128 * 128;         // weight tile: 128 rows x 128 bytes
 constexpr int kSFStep = 512;              // one operand's scales for one MMA: 32 rows x 16 B
 constexpr int kSFBytes = kKSteps * kSFStep;
+constexpr int kSFRaw = 128 * (kKC / 16);  // one stage's weight scales, row-major
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kDcol = 0;             // D: two buffers of kTS columns
 
 // Sizes for TS tokens per pass: 128 (many tokens per expert), or 64 -- a
 // smaller token tile leaves room for two more stages, i.e. more weight
 // bytes in flight per SM, which experts with few tokens need.
-template <int TS>
+template <int TS, bool SFT>
 struct Cfg {
   static constexpr int kTS = TS;                        // tokens per pass (MMA N <= TS)
   static constexpr int kStages = TS >= 128 ? 5 : 7;
   static constexpr int kBTile = TS * 128;               // token tile: TS rows x 128 bytes
-  static constexpr int kStageBytes = kATile + kBTile + 2 * kSFBytes;
+  // weight tile, token tile, both operands' scales in the tensor core's layout,
+  // and (SFT) the weight scales as the TMA lands them (128 rows x 16 bytes)
+  static constexpr int kSFRawBytes = SFT ? kSFRaw : 0;
+  static constexpr int kStageBytes = kATile + kBTile + 2 * kSFBytes + kSFRawBytes;
   static constexpr uint32_t kSFcol = 2 * TS;            // per stage: 16 columns of A scales, 16 of B
   static constexpr size_t kOffStart = (size_t)kStages * kStageBytes;
   static constexpr size_t kOffEid = kOffStart + (kMaxExperts + 4) * 4;
@@ -112,10 +120,14 @@ struct UnitWalk {
   }
 };
 
-template <int TS>
+// SFT: the weight scales arrive by TMA with the weight tile (row-major) and
+// the staging warps move them into the tensor core's scale layout (K % 256
+// == 0: 16-byte scale rows); otherwise they are gathered 4 bytes at a time.
+template <int TS, bool SFT>
 __global__ void __launch_bounds__(kThreads, 1)
-    grouped_gemv_bs_kernel(const Params p, const __grid_constant__ CUtensorMap tmap_w) {
-  using C = Cfg<TS>;
+    grouped_gemv_bs_kernel(const Params p, const __grid_constant__ CUtensorMap tmap_w,
+                           const __grid_constant__ CUtensorMap tmap_sfw) {
+  using C = Cfg<TS, SFT>;
   constexpr int kTS = C::kTS, kStages = C::kStages, kBTile = C::kBTile;
   constexpr int kStageBytes = C::kStageBytes;
   constexpr uint32_t kSFcol = C::kSFcol;
@@ -154,7 +166,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == kProdWarp && lane == 0) prefetch_tmap(&tmap_w);
+  if (warp == kProdWarp && lane == 0) {
+    prefetch_tmap(&tmap_w);
+    if (SFT) prefetch_tmap(&tmap_sfw);
+  }
   if (warp == kMmaWarp) tmem_alloc(tmem_slot, kTmemCols);
   pdl_wait();
   pdl_launch_dependents();
@@ -196,8 +211,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int s = (int)(it % kStages);
           wait(&empty[s], ((it / kStages) & 1u) ^ 1u);
           if (*abort_flag) break;
-          mbar_arrive_expect_tx(&a_full[s], (uint32_t)kATile);
+          mbar_arrive_expect_tx(&a_full[s], (uint32_t)(kATile + (SFT ? kSFRaw : 0)));
           tma_load_3d(stage(s), &tmap_w, c * (kKC / 2), r.n0, r.e, &a_full[s], policy);
+          if (SFT)  // 128 rows x the stage's 16 scale bytes; rows past N, columns past K: zeros
+            tma_load_3d(stage(s) + kStageBytes - kSFRaw, &tmap_sfw, c * (kKC / 16), r.n0, r.e,
+                        &a_full[s], policy);
           issued = it + 1;
         }
       }
@@ -338,9 +356,23 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               const int off = skk * kSFStep + sr0 * 16 + i * 4;  // row sr0 + 32 i of the layout
-              if (arow[i] >= 0) cp_async4_zfill(sfa_s + off, p.sfw + arow[i] + kc, 4u);
+              if (!SFT && arow[i] >= 0) cp_async4_zfill(sfa_s + off, p.sfw + arow[i] + kc, 4u);
               if (srow[i] >= 0) cp_async4_zfill(sfb_s + off, p.sfa + srow[i] + kc, 4u);
             }
+          }
+          if (SFT) {
+            // weight row t's 16 scale bytes (one word per MMA k-step), from the
+            // TMA's row-major box into row t of each k-step's 32 x 16-byte atom
+            wait(&a_full[s], (it / kStages) & 1u);
+            if (!*abort_flag) {
+              const uint4 v = *reinterpret_cast<const uint4 *>(stage(s) + kStageBytes - kSFRaw + t * 16);
+              const int off = (t & 31) * 16 + (t >> 5) * 4;
+              *reinterpret_cast<uint32_t *>(sfa_s + 0 * kSFStep + off) = v.x;
+              *reinterpret_cast<uint32_t *>(sfa_s + 1 * kSFStep + off) = v.y;
+              *reinterpret_cast<uint32_t *>(sfa_s + 2 * kSFStep + off) = v.z;
+              *reinterpret_cast<uint32_t *>(sfa_s + 3 * kSFStep + off) = v.w;
+            }
+            fence_proxy_async_smem();  // plain stores, read by tcgen05.cp
           }
         }
         cp_async_mbar_arrive_noinc(&b_full[s]);

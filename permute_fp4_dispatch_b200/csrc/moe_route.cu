@@ -183,6 +183,7 @@ struct LibMaps {
                         // and the line map of the decode variant
   CUtensorMap tw, tsf, tlines, tsf_lines;
   CUtensorMap tbs;      // block-scaled variant: 128 rows x 128 bytes, 128B swizzle
+  CUtensorMap tbs_sf;   // and its weight scales: 128 rows x 16 bytes (K % 256 == 0)
 };
 constexpr int kMapCache = 8;
 LibMaps g_maps[kMapCache];
@@ -207,6 +208,7 @@ bool library_maps(const uint8_t *w, const uint8_t *sfw, int E, int N, int K, Lib
   std::memset(&m.tlines, 0, sizeof m.tlines);
   std::memset(&m.tsf_lines, 0, sizeof m.tsf_lines);
   std::memset(&m.tbs, 0, sizeof m.tbs);
+  std::memset(&m.tbs_sf, 0, sizeof m.tbs_sf);
   // the tensor-memory variant reads 16-row x 128-byte weight boxes and 16-row x 16-byte scale boxes
   static_assert(moe::gemv::tc::kWStride == 128 && moe::gemv::tc::kSFStride == 16, "box width");
   if (!encode_u8_3d(&m.tw, w, (uint64_t)K / 2, (uint64_t)N, (uint64_t)E, 128, 16,
@@ -217,6 +219,9 @@ bool library_maps(const uint8_t *w, const uint8_t *sfw, int E, int N, int K, Lib
                     CU_TENSOR_MAP_SWIZZLE_128B))
     return false;
   if (m.sf_tma && !encode_u8_3d(&m.tsf, sfw, (uint64_t)K / 16, (uint64_t)N, (uint64_t)E, 16, 16,
+                                CU_TENSOR_MAP_SWIZZLE_NONE))
+    return false;
+  if (m.sf_tma && !encode_u8_3d(&m.tbs_sf, sfw, (uint64_t)K / 16, (uint64_t)N, (uint64_t)E, 16, 128,
                                 CU_TENSOR_MAP_SWIZZLE_NONE))
     return false;
   if (m.sf_tma && !encode_lines_4d(&m.tlines, w, (uint64_t)K, (uint64_t)N, (uint64_t)E,
@@ -690,11 +695,19 @@ moe_status_t moe_grouped_gemv_nvfp4(moe_gemv_mode_t mode, const void *act, const
     // passes of 64 tokens (two more stages in flight) when the experts hold
     // 64 tokens or fewer on average, else 128
     const bool small = S <= (int64_t)64 * E;
-    void (*kern)(const Params, const CUtensorMap) =
-        small ? bs::grouped_gemv_bs_kernel<64> : bs::grouped_gemv_bs_kernel<128>;
-    const size_t smem = small ? bs::Cfg<64>::kSmemBytes : bs::Cfg<128>::kSmemBytes;
+    // weight scales by TMA when their rows are whole 16-byte units (K % 256 == 0)
+    void (*kern)(const Params, const CUtensorMap, const CUtensorMap) =
+        small ? (maps.sf_tma ? bs::grouped_gemv_bs_kernel<64, true>
+                             : bs::grouped_gemv_bs_kernel<64, false>)
+              : (maps.sf_tma ? bs::grouped_gemv_bs_kernel<128, true>
+                             : bs::grouped_gemv_bs_kernel<128, false>);
+    const size_t smem = small ? (maps.sf_tma ? bs::Cfg<64, true>::kSmemBytes
+                                             : bs::Cfg<64, false>::kSmemBytes)
+                              : (maps.sf_tma ? bs::Cfg<128, true>::kSmemBytes
+                                             : bs::Cfg<128, false>::kSmemBytes);
     if ((st = set_smem(kern, smem)) != MOE_OK) return st;
-    return launch_pdl(kern, dim3((unsigned)sms), dim3(bs::kThreads), smem, s, p, maps.tbs);
+    return launch_pdl(kern, dim3((unsigned)sms), dim3(bs::kThreads), smem, s, p, maps.tbs,
+                      maps.tbs_sf);
   }
   if (use_mma) {
     void (*kern)(const Params, const int, const CUtensorMap, const CUtensorMap) =
