@@ -10,7 +10,11 @@
 // Design (taken when experts hold more tokens than a decode pass; the FP4
 // weight stream and its dequantisation bound it):
 //   * Work is expert-major: an active expert's pairs (CSR from
-//     moe_create_indices) are taken in passes of up to kTS = 64 tokens and
+//     moe_create_indices) are taken in passes of up to kTS = 64 tokens (128
+//     for W4A16 whose activations were converted once per call, when the
+//     experts hold more than 64 tokens on average: the token tile then
+//     arrives by cp.async straight from the converted rows, one item ahead,
+//     and each pass dequantises the weights for twice the tokens) and
 //     each pass sweeps the expert's N rows in 16-row blocks.  The flat list of
 //     (expert, pass, row block) units is split into equal contiguous ranges
 //     cut at round boundaries, one per persistent CTA (grid = SM count).
@@ -59,31 +63,40 @@ constexpr int kTmaWarp = kDQ;
 constexpr int kMmaWarp = kDQ + 1;
 constexpr int kThreads = (kDQ + 2) * 32;
 constexpr int kKC = 256;                // columns (codes) per chunk
-constexpr int kTS = 64;                 // tokens per pass (MMA N <= 64)
-constexpr int kStages = 5;
 constexpr int kWStride = kKC / 2;       // bytes per weight row in a stage (128B-swizzled)
 constexpr int kSFStride = kKC / 16;     // bytes per scale row in a stage
 constexpr int kBoxW = 16 * kWStride;    // one 16-row weight box
 constexpr int kBoxSF = 16 * kSFStride;  // one 16-row scale box
 constexpr int kStageW = 128 * kWStride;
 constexpr int kStageBytes = kStageW + 128 * kSFStride;
-constexpr int kKatomBytes = kTS * 128;  // one 64-column slab of the B tile
-constexpr int kBTile = 4 * kKatomBytes;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAcol = 0;           // A tiles: columns [0, 256), 128 per buffer
-constexpr uint32_t kDcol = 256;         // D tiles: columns [256, 384), 64 per buffer
-
+constexpr uint32_t kDcol = 256;         // D tiles: two buffers of kTS columns from 256
 static_assert(kStageBytes % 1024 == 0, "stages must keep the 1024-byte swizzle alignment");
-constexpr size_t kOffB = (size_t)kStages * kStageBytes;
-constexpr size_t kOffPrefix = kOffB + 2 * kBTile;
-constexpr size_t kOffStart = kOffPrefix + (kMaxExperts + 4) * 4;
-constexpr size_t kOffEid = kOffStart + (kMaxExperts + 4) * 4;
-constexpr size_t kOffPair = kOffEid + (kMaxExperts + 4) * 4;     // [2][kTS] pair ids
-constexpr size_t kOffShift = kOffPair + 2 * kTS * 4;  // [2][kTS] W4A16 token offsets
-constexpr size_t kOffBar = kOffShift + 2 * kTS * 4;
-constexpr int kNumBars = 2 * kStages + 9;
-constexpr size_t kOffMisc = kOffBar + kNumBars * 8;             // tmem slot, abort flag
-constexpr size_t kSmemBytes = kOffMisc + 16 + 1024;             // + alignment slack
+
+// Sizes for TS tokens per pass (MMA N <= TS): 64, or 128 for W4A16 whose
+// activations were converted once per call (the token tile then arrives by
+// cp.async straight from the converted rows, and a pass of 128 tokens
+// halves the weight dequantisation per token).
+template <int TS>
+struct Cfg {
+  static constexpr int kTS = TS;
+  static constexpr int kStages = TS >= 128 ? 4 : 5;
+  static constexpr int kKatomBytes = TS * 128;  // one 64-column slab of the B tile
+  static constexpr int kBTile = 4 * kKatomBytes;
+  static constexpr size_t kOffB = (size_t)kStages * kStageBytes;
+  static constexpr size_t kOffPrefix = kOffB + 2 * kBTile;
+  static constexpr size_t kOffStart = kOffPrefix + (kMaxExperts + 4) * 4;
+  static constexpr size_t kOffEid = kOffStart + (kMaxExperts + 4) * 4;
+  static constexpr size_t kOffPair = kOffEid + (kMaxExperts + 4) * 4;  // [2][kTS] pair ids
+  static constexpr size_t kOffShift = kOffPair + 2 * TS * 4;           // [2][kTS] token offsets
+  static constexpr size_t kOffBar = kOffShift + 2 * TS * 4;
+  static constexpr int kNumBars = 2 * kStages + 9;
+  static constexpr size_t kOffMisc = kOffBar + kNumBars * 8;            // tmem slot, abort flag
+  static constexpr size_t kSmemBytes = kOffMisc + 16 + 1024;            // + alignment slack
+  static_assert(kDcol + 2 * TS <= kTmemCols, "tensor memory columns");
+  static_assert(kSmemBytes <= 232448, "shared memory per block");
+};
 
 // W4A16 activations converted once per call for this variant (it stages
 // activations for every 128-row round and 256-column chunk, so converting
@@ -136,11 +149,20 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-template <int MODE, bool SF_TMA>
+template <int MODE, bool SF_TMA, int TS>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemv_kernel(const Params p, const __grid_constant__ CUtensorMap tmap_w,
                         const __grid_constant__ CUtensorMap tmap_sf,
                         const uint16_t *__restrict__ act16, const int32_t *__restrict__ act_shift) {
+  using C = Cfg<TS>;
+  constexpr int kTS = C::kTS, kStages = C::kStages, kKatomBytes = C::kKatomBytes;
+  constexpr int kBTile = C::kBTile;
+  constexpr size_t kOffB = C::kOffB, kOffPrefix = C::kOffPrefix, kOffStart = C::kOffStart;
+  constexpr size_t kOffEid = C::kOffEid, kOffPair = C::kOffPair, kOffShift = C::kOffShift;
+  constexpr size_t kOffBar = C::kOffBar, kOffMisc = C::kOffMisc;
+  constexpr int kTPW = TS / 8;  // tokens per staging warp: lane i < kTPW holds token warp + 8 i
+  // the 128-token form reads converted activations only (the host picks it so)
+  static_assert(TS == 64 || MODE == MOE_W4A16, "128-token passes take converted W4A16 rows");
   pdl_wait();
   pdl_launch_dependents();
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -280,7 +302,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const int nmma = (r.ntok + 15) / 16 * 16;
         const uint32_t idesc = umma_idesc_f16(128, nmma);
-        const uint32_t d_t = tbase + kDcol + d * 64u;
+        const uint32_t d_t = tbase + kDcol + d * (uint32_t)kTS;
         for (int c = 0; c < nchunks; ++c, ++it) {
           const uint32_t b = it & 1u;
           wait(&a_full[b], (it >> 1) & 1u);
@@ -318,14 +340,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool have_n = have && iter.next(meta, RB, rn);
     bool ep_pending = false;
     uint32_t it = 0, rnd = 0, rnd_p = 0;
-    // token pair ids of the current / next round, one token per lane (lanes < 8):
-    // lane i of warp w holds token tau = w + 8 i
+    // token pair ids of the current / next round, one token per lane (lanes <
+    // kTPW): lane i of warp w holds token tau = w + 8 i
     uint32_t pair_cur = 0xFFFFFFFFu, pair_nxt = 0xFFFFFFFFu;
     int32_t sh_cur = 0, sh_nxt = 0;  // the same tokens' W4A16 offsets (0 without act16)
     const bool pre = MODE == MOE_W4A16 && act16 != nullptr;  // activations converted already
     auto fetch_pairs = [&](const Round &q_, uint32_t &dst, int32_t &sh) {
       const int tau = warp + 8 * lane;
-      dst = (lane < 8 && tau < q_.ntok) ? p.order[q_.tok0 + tau] : 0xFFFFFFFFu;
+      dst = (lane < kTPW && tau < q_.ntok) ? p.order[q_.tok0 + tau] : 0xFFFFFFFFu;
       sh = (pre && dst != 0xFFFFFFFFu) ? act_shift[dst / (uint32_t)p.top_k] : 0;
     };
     if (have) fetch_pairs(r, pair_cur, sh_cur);
@@ -353,26 +375,47 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     };
-    if (have) load_act(pair_cur, r.ntok, 0);
+    // (128-token passes) the converted rows of this warp's tokens for one chunk,
+    // copied straight into B buffer bb: 16 bytes per lane and token
+    auto copy_act = [&](uint32_t pairs, int ntok, int c, uint32_t bb) {
+      const int k0 = c * kKC;
+      const int kcb = min(kKC, K - k0);
+      const bool kv = 8 * lane < kcb;
+      uint8_t *bt = btile + bb * kBTile;
+      const int katom = lane >> 3, cidx = lane & 7;
+#pragma unroll
+      for (int i = 0; i < kTPW; ++i) {
+        const uint32_t pr = __shfl_sync(0xffffffffu, pairs, i);
+        const int tau = warp + 8 * i;
+        if (tau < ntok && kv)
+          cp_async16_zfill(bt + katom * kKatomBytes + tau * 128 + ((cidx ^ (tau & 7)) * 16),
+                           act16 + (int64_t)(pr / (uint32_t)p.top_k) * K + k0 + 8 * lane, 16u);
+      }
+    };
+    if constexpr (TS < 128) {
+      if (have) load_act(pair_cur, r.ntok, 0);
+    } else {
+      if (have) copy_act(pair_cur, r.ntok, 0, 0u);  // buffer 0 has no earlier user
+    }
 
     auto epilogue = [&](const Round &er, uint32_t ernd) {
       const uint32_t d = ernd & 1u;
       wait(&d_full[d], (ernd >> 1) & 1u);
       tc_fence_after();
-      const int c0 = 32 * h;  // this warp's token columns
-      uint32_t v[32];
+      constexpr int kCols = kTS / 2;  // this warp's token columns: kCols from kCols * h
+      const int c0 = kCols * h;
+      uint32_t v[kCols];
       const bool cols = c0 < er.ntok && 32 * q < er.nrows;
       if (cols) {
-        uint32_t t0[16], t1[16];
-        const uint32_t ta = tbase + lane_base + kDcol + d * 64u + (uint32_t)c0;
-        tmem_ld16(ta, t0);
-        tmem_ld16(ta + 16u, t1);
+        uint32_t t[kCols / 16][16];
+        const uint32_t ta = tbase + lane_base + kDcol + d * (uint32_t)kTS + (uint32_t)c0;
+#pragma unroll
+        for (int j = 0; j < kCols / 16; ++j) tmem_ld16(ta + 16u * (uint32_t)j, t[j]);
         tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          v[i] = t0[i];
-          v[16 + i] = t1[i];
-        }
+        for (int j = 0; j < kCols / 16; ++j)
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[16 * j + i] = t[j][i];
       }
       tc_fence_before();
       __syncwarp();
@@ -383,9 +426,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int n = er.n0 + row;
         const uint32_t *pairs = s_pair + (ernd & 1u) * kTS;
         const int32_t *shifts = s_shift + (ernd & 1u) * kTS;
-        const int ncol = min(32, er.ntok - c0);
+        const int ncol = min(kCols, er.ntok - c0);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
+        for (int i = 0; i < kCols; ++i) {
           if (i < ncol) {
             const uint32_t pr = pairs[c0 + i];
             float y = __fmul_rn(__uint_as_float(v[i]), f);
@@ -403,7 +446,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     while (have) {
       // ---- round start: publish this round's pair ids, fetch the next round's
       named_bar_sync(1, kDQ * 32);
-      if (lane < 8 && warp + 8 * lane < r.ntok) {
+      if (lane < kTPW && warp + 8 * lane < r.ntok) {
         s_pair[(rnd & 1u) * kTS + warp + 8 * lane] = pair_cur;
         s_shift[(rnd & 1u) * kTS + warp + 8 * lane] = sh_cur;
       }
@@ -455,11 +498,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_st16(tbase + lane_base + kAcol + b * 128u + 64u * (uint32_t)h + 16u * (uint32_t)jj, rr);
           }
         }
-        // ---- activations of this chunk -> fp16 B tile (K-major, 128B swizzle)
+        // ---- activations of this chunk -> fp16 B tile (K-major, 128B swizzle);
+        // with 128-token passes it was copied in during the previous item
         uint8_t *bt = btile + b * kBTile;
         unsigned range_bad = 0;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
+        for (int i = 0; i < (TS < 128 ? 8 : 0); ++i) {
           const int tau = warp + 8 * i;
           if (tau >= r.ntok) continue;  // warp-uniform
           uint4 hv;
@@ -490,11 +534,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           *reinterpret_cast<uint4 *>(bt + katom * kKatomBytes + tau * 128 + ((cidx ^ (tau & 7)) * 16)) = hv;
         }
         if (MODE == MOE_W4A16 && range_bad) raise_device_error(MOE_DEVERR_ACT_RANGE);
-        // prefetch the next chunk's activations (or the next round's first chunk)
-        if (c + 1 < nchunks) {
-          load_act(pair_cur, r.ntok, c + 1);
-        } else if (have_n) {
-          load_act(pair_nxt, rn.ntok, 0);
+        if constexpr (TS < 128) {
+          // prefetch the next chunk's activations (or the next round's first chunk)
+          if (c + 1 < nchunks) {
+            load_act(pair_cur, r.ntok, c + 1);
+          } else if (have_n) {
+            load_act(pair_nxt, rn.ntok, 0);
+          }
+        } else {
+          cp_async_wait_all();  // this item's token tile, copied in during the previous item
         }
         // ---- publish A (TMEM) and B (shared memory) of item it; release stage s
         tmem_wait_st();
@@ -504,6 +552,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
           mbar_arrive(&empty[s]);
           mbar_arrive(&a_full[b]);
+        }
+        if constexpr (TS >= 128) {
+          // the next item's token tile into the other buffer, once the MMAs of
+          // item it - 1, its previous user, are done
+          const uint32_t bn = (it + 1) & 1u;
+          if (it >= 1) wait(&a_empty[bn], ((it - 1) >> 1) & 1u);
+          if (!*abort_flag) {
+            if (c + 1 < nchunks)
+              copy_act(pair_cur, r.ntok, c + 1, bn);
+            else if (have_n)
+              copy_act(pair_nxt, rn.ntok, 0, bn);
+          }
         }
         // ---- the previous round's epilogue overlaps this round's first chunk
         if (c == 0 && ep_pending) {
@@ -522,6 +582,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       have_n = have && iter.next(meta, RB, rn);
     }
     if (ep_pending) epilogue(rp, rnd_p);
+    cp_async_wait_all();  // no token-tile copy may still land after the CTA exits
   }
 
   tc_fence_before();

@@ -724,14 +724,21 @@ moe_status_t moe_grouped_gemv_nvfp4(moe_gemv_mode_t mode, const void *act, const
   }
   void (*kern)(const Params, const CUtensorMap, const CUtensorMap, const uint16_t *,
                const int32_t *);
-  if (mode == MOE_W4A16)
-    kern = maps.sf_tma ? tc::grouped_gemv_kernel<MOE_W4A16, true>
-                       : tc::grouped_gemv_kernel<MOE_W4A16, false>;
+  // passes of 128 tokens when the activations were converted and the experts
+  // hold more than 64 tokens on average, else 64
+  const bool wide = a16.act16 != nullptr && S > (int64_t)64 * E;
+  if (mode == MOE_W4A16 && wide)
+    kern = maps.sf_tma ? tc::grouped_gemv_kernel<MOE_W4A16, true, 128>
+                       : tc::grouped_gemv_kernel<MOE_W4A16, false, 128>;
+  else if (mode == MOE_W4A16)
+    kern = maps.sf_tma ? tc::grouped_gemv_kernel<MOE_W4A16, true, 64>
+                       : tc::grouped_gemv_kernel<MOE_W4A16, false, 64>;
   else
-    kern = maps.sf_tma ? tc::grouped_gemv_kernel<MOE_W4A4, true>
-                       : tc::grouped_gemv_kernel<MOE_W4A4, false>;
-  if ((st = set_smem(kern, tc::kSmemBytes)) != MOE_OK) return st;
-  return launch_pdl(kern, dim3((unsigned)sms), dim3(tc::kThreads), tc::kSmemBytes, s, p, maps.tw,
+    kern = maps.sf_tma ? tc::grouped_gemv_kernel<MOE_W4A4, true, 64>
+                       : tc::grouped_gemv_kernel<MOE_W4A4, false, 64>;
+  const size_t smem = wide ? tc::Cfg<128>::kSmemBytes : tc::Cfg<64>::kSmemBytes;
+  if ((st = set_smem(kern, smem)) != MOE_OK) return st;
+  return launch_pdl(kern, dim3((unsigned)sms), dim3(tc::kThreads), smem, s, p, maps.tw,
                     maps.tsf, static_cast<const uint16_t *>(a16.act16),
                     static_cast<const int32_t *>(a16.shift));
 }

@@ -305,6 +305,10 @@ GEMV_CASES = [
                                      N_out=264), "w4a16"),
     ("passes-w4a4", wl.small_config("passes", N=300, real=290, K=512, E=4, top_k=2,
                                     N_out=264), "w4a4"),
+    # 128-token passes of the tensor-memory variant with a ragged last chunk
+    # (544 = 2 x 256 + 32) and gathered scale rows
+    ("passes-ragged-k", wl.small_config("passes_rk", N=300, real=290, K=544, E=4, top_k=2,
+                                        N_out=136), "w4a16"),
     # minimal K, N
     ("minimal", wl.small_config("minimal", N=3, real=3, K=64, E=2, top_k=1, N_out=8), "w4a16"),
     # K % 256 == 0 with a partial last stage of 1024 columns (2304 = 2 x 1024 + 256),
