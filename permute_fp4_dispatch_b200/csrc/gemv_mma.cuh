@@ -34,9 +34,10 @@
 //     4 * row + line, so the swizzle key is (row & 1) * 4 + line and the eight
 //     lanes of one shared-memory phase (rows g, g + 1) hit eight distinct
 //     16-byte bank groups.
-//   * Every pair requests its first stage as soon as the CTA knows its
-//     range, so the weights stream while the CTA compacts its token lists
-//     and builds its first activation tile.
+//   * The CTA requests its first pass's activation rows as soon as its token
+//     lists are compacted, and every pair its first weight stage right
+//     after, so the rows do not queue behind the weights' first burst and
+//     the weights stream while the CTA converts its first activation tile.
 //   * When a CTA starts a new (expert, pass), it builds that pass's fp16
 //     activation tile once, for the whole K; every round of the pass reuses
 //     it.  The tile is token-major, one row per token: W4A16 rows arrive as
@@ -418,9 +419,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     ++produced;
     if (++pc == nst) next_own_round();
   };
-  // the first stage of every pair is requested as soon as the range is known:
-  // the weights stream while the CTA gathers its token lists and activations
-  produce();
 
   uint32_t *s_passes = reinterpret_cast<uint32_t *>(smem + kOffPasses);
   int n_passes = 0;
@@ -502,6 +500,29 @@ __global__ void __launch_bounds__(kThreads, 1)
   RoundWalk iter;
   iter.init(meta, A, RB, u_begin, u_end);
   Round r;
+  // W4A16: the first pass's activation rows are requested before any weight
+  // stage, so they do not wait behind the weight stream's first burst
+  const bool first_rows_early = MODE == MOE_W4A16;
+  if (first_rows_early && warp == 0) {
+    RoundWalk peek = iter;
+    Round r0;
+    if (peek.next(meta, RB, (uint32_t)ts, r0)) {
+      uint32_t row0 = 0;
+      if (lane < r0.ntok)
+        row0 = (fused ? s_passes[lane] : __ldg(p.order + r0.tok0 + lane)) / (uint32_t)p.top_k;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(act_bar, (uint32_t)r0.ntok * (uint32_t)K * 2u);
+        ++act_issued;
+      }
+      __syncwarp();
+      if (lane < r0.ntok)
+        bulk_load_g2s(act + lane * arow, static_cast<const uint16_t *>(p.act) + (int64_t)row0 * K,
+                      (uint32_t)K * 2u, act_bar);
+    }
+  }
+  __syncthreads();  // the first rows are requested before every pair's first weight stage
+  // then the weights stream while the CTA converts its first activation tile
+  produce();
   uint32_t consumed = 0;
   uint32_t pass_key = 0xFFFFFFFFu;
   int ng = 0;
@@ -530,7 +551,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // the previous tile is free once every warp is here
         if (pass_key != 0xFFFFFFFFu) named_bar_sync(1, kThreads);
         // each token's bf16 row, one bulk copy straight into its tile row
-        if (warp == 0 && !__shfl_sync(0xFFFFFFFFu, *abort_flag, 0)) {
+        if (warp == 0 && !(pass_idx == 0 && first_rows_early) &&
+            !__shfl_sync(0xFFFFFFFFu, *abort_flag, 0)) {
           // the previous pass's plain reads and writes of the tile come before
           // the copies' writes
           fence_proxy_async_smem();
