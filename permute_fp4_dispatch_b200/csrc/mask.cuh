@@ -12,11 +12,16 @@ namespace moe {
 
 // Grid-stride over the masked tail of the flattened [N, top_k] map.  The
 // masked region is a contiguous suffix, so each thread writes whole int64
-// slots with no per-row test.
+// slots with no per-row test.  The next grid in the stream may be scheduled
+// at once: the kernels of this library that follow it run their input-free
+// set-up (barriers, descriptor and L2 prefetches) meanwhile and read the map
+// only after their own wait for this grid's completion.
 __global__ void __launch_bounds__(256) mask_padding_kernel(int64_t *__restrict__ map, int32_t N,
                                                            int32_t top_k,
                                                            const int32_t *__restrict__ real_ptr,
                                                            int32_t tp_rank) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int64_t real = static_cast<int64_t>(*real_ptr);
   int64_t first = real - static_cast<int64_t>(tp_rank) * N;  // first masked local row
   first = first < 0 ? 0 : (first > N ? N : first);

@@ -283,9 +283,8 @@ moe_status_t moe_mask_padding(int64_t *routing_map, int32_t N, int32_t top_k,
   const int64_t slots = (int64_t)N * top_k;
   int64_t blocks = (slots + 255) / 256;
   if (blocks > (int64_t)sms * 8) blocks = (int64_t)sms * 8;
-  moe::mask_padding_kernel<<<(unsigned)blocks, 256, 0, s>>>(routing_map, N, top_k,
-                                                             real_token_count, tp_rank);
-  return launch_status();
+  return launch_pdl(moe::mask_padding_kernel, dim3((unsigned)blocks), dim3(256), 0, s, routing_map,
+                    N, top_k, real_token_count, tp_rank);
 }
 
 // ------------------------------------------------------------------ step 2
